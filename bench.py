@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Benchmark of libfattn on B200: one JSON line on stdout (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the prefill hot path (closed-form KV tile ranges, TMA
+Q/K/V tiles, tcgen05 S = Q K^T, masked exp2 online softmax, P V, O / l and
+LSE) over the causal 4 x 16 x 4096, d = 128 bf16 workload; ``value`` is its
+in-mask TFLOP/s (4 d FLOPs per allowed (q, k) pair per head) with inputs
+resident in HBM.  The same run times the split-KV decode path (split kernel +
+LSE merge) on the 64 x 32 x 32768 cache and reports it under ``decode`` in
+GB/s of K/V/q/o/lse traffic, and the sliding-window / long-causal prefill
+workloads under ``extra``.
+
+Multi-GPU (torchrun, one rank per GPU): (batch, head) units are independent,
+so every rank runs its own full copy of the workload with no collective on the
+data path (weak scaling); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+HEADLINE = "causal_4k"
+DECODE = "decode_32k"
+EXTRA = ["window_bidir_32k", "window_causal_32k", "causal_64k_qscale"]
+PREFILL_KERNEL = "attn_fwd_sm100_kernel"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "io_aware_exact_34_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    ent = rec.get(kernel, {}).get(workload)
+    if not ent or ent.get("source_digest") != kernel_source_digest():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed regions."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, busy_power_w=300.0):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"]}
+        busy = [r for r in rows if r[2] >= busy_power_w] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in busy for i, flag in enumerate(r[3]) if flag.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in busy), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(busy), "power_w_max": max(r[2] for r in rows), "reasons": reasons}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value: float) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed(world, fn, steps, warmup):
+    """Average device ms per step of fn over `steps`, CUDA events on the
+    current stream, barrier + synchronize on both sides, max over ranks."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        fn()
+    end.record()
+    end.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(world, start.elapsed_time(end) / steps)
+
+
+def prefill_flops(fl, w):
+    c = fl.attn_count_blocks(w.Lq, w.Lk, w.causal, w.window_left, w.window_right, 128, 128)
+    return 4.0 * w.d * c["pairs"] * w.B * w.H, c
+
+
+def cpu_baseline_sample(w, budget_s=12.0):
+    """The oracle, as it stands, on whole heads of the workload until about
+    `budget_s` seconds of work have run on all host cores."""
+    from io_aware_exact_34_b200 import synth
+    from oracle import oracle
+    oracle.build()
+    q, k, v = synth.make_inputs(w)
+    import torch
+    pairs_per_head = None
+    flops = 0.0
+    heads = 0
+    t0 = time.perf_counter()
+    for bh in range(w.B * w.H):
+        b, h = divmod(bh, w.H)
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        oracle.attn(q[sl], k[sl], v[sl], w.scale, w.causal, w.window_left, w.window_right)
+        if pairs_per_head is None:
+            c = oracle.count_blocks(w.Lq, w.Lk, w.causal, w.window_left, w.window_right, 128, 128)
+            pairs_per_head = c["pairs"]
+        flops += 4.0 * w.d * pairs_per_head
+        heads += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    del torch
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{heads} of {w.B * w.H} (b,h) heads of {w.name}, every row, fp64, {dt:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    """The oracle timed on the host cores (the reference arm of this build)."""
+    if rank != 0:
+        return
+    from io_aware_exact_34_b200 import synth
+    from oracle import oracle
+    oracle.build()
+    w = synth.WORKLOADS[HEADLINE]
+    q, k, v = synth.make_inputs(w)
+    rows_per_step = 256
+    g_rows = synth.sample_rows(w, n_random=0, seed=0, full_heads=[(w.B - 1, w.H - 1)]).numpy()
+    g_rows = g_rows[g_rows[:, 0] == w.B - 1]
+    g_rows = g_rows[g_rows[:, 1] == w.H - 1]
+    # each step: 256 consecutive rows of the last head (every allowed key of each)
+    def step(s):
+        lo = (s * rows_per_step) % w.Lq
+        rows = g_rows[lo:lo + rows_per_step]
+        oracle.attn_rows(q, k, v, rows, w.scale, w.causal, w.window_left, w.window_right)
+        i = rows[:, 2]
+        return float(4.0 * w.d * (i + 1).sum())  # causal: row i has i + 1 keys
+    for s in range(args.warmup):
+        step(s)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for s in range(args.steps):
+        flops += step(args.warmup + s)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    line = {"metric": "attention fwd TFLOP/s (in-mask FLOPs)", "value": value, "unit": "TFLOP/s",
+            "impl": "reference", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {**w.describe(), "parallelism": "oracle on host cores"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"{rows_per_step} consecutive query rows of head (b,h)=({w.B - 1},{w.H - 1}) per step"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    from io_aware_exact_34_b200 import fattn, synth
+    peaks, peak_src = load_peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    # ---------------------------------------------------------------- headline prefill
+    w = synth.WORKLOADS[HEADLINE]
+    flops, counts = prefill_flops(fattn, w)
+    q, k, v = synth.make_inputs(w, device=dev, seed=w.seed + rank)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev)
+
+    def step():
+        fattn.attn_fwd(q, k, v, o=o, lse=lse, scale=w.scale, causal=w.causal,
+                       window_left=w.window_left, window_right=w.window_right)
+
+    with ClockSampler(local) as clk:
+        ms = timed(world, step, args.steps, args.warmup)
+        # keep the same work running for about a second so the sampler sees it
+        t_end = time.perf_counter() + 1.0
+        while time.perf_counter() < t_end:
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize()
+    clocks = clk.summary()
+
+    value = world * flops / (ms * 1e-3) / 1e12
+    achieved = flops / (ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": recorded_traffic(PREFILL_KERNEL, w.name),
+                "peak_source": f"{peak_src} bf16 dense (burst)", "kernel": PREFILL_KERNEL}
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+        oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            fattn.attn_fwd(qd, kd, vd, o=o, lse=lse, scale=w.scale, causal=w.causal,
+                           window_left=w.window_left, window_right=w.window_right)
+            oh.copy_(o, non_blocking=True)
+            lh.copy_(lse, non_blocking=True)
+
+        ms_e2e = timed(world, e2e_step, max(3, args.steps // 4), min(args.warmup, 3))
+        e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": int(3 * q.numel() * q.element_size()),
+               "d2h_bytes_per_step": int(o.numel() * o.element_size() + lse.numel() * 4)}
+        del qh, kh, vh, oh, lh, qd, kd, vd
+
+    # ---------------------------------------------------------------- decode
+    decode = None
+    if not args.no_decode:
+        wd = synth.WORKLOADS[DECODE]
+        dq, dk, dv = synth.make_inputs(wd, device=dev, seed=wd.seed + rank)
+        do = torch.empty_like(dq)
+        dl = torch.empty((wd.B, wd.H), dtype=torch.float32, device=dev)
+        ws = torch.empty(fattn.attn_decode_workspace_bytes(wd.B, wd.H, wd.Lk, wd.d, wd.num_splits),
+                         dtype=torch.uint8, device=dev)
+
+        def dstep():
+            fattn.attn_decode_splitkv(dq, dk, dv, o=do, lse=dl, scale=wd.scale, num_splits=wd.num_splits,
+                                      workspace=ws)
+
+        dsteps = max(5, min(args.steps, 40))
+        dms = timed(world, dstep, dsteps, max(3, min(args.warmup, 5)))
+        dbytes = (dk.numel() + dv.numel() + dq.numel() + do.numel()) * 2 + dl.numel() * 4
+        gbs = dbytes / (dms * 1e-3) / 1e9
+        decode = {"metric": "decode HBM GB/s", "value": world * gbs, "unit": "GB/s", "ms_per_step": dms,
+                  "steps": dsteps, "config": wd.describe(),
+                  "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": gbs / peaks["hbm_gbs"], "traffic": recorded_traffic("decode_split_kernel", wd.name),
+                               "peak_source": f"{peak_src} copy bandwidth",
+                               "kernels": ["decode_split_kernel", "decode_merge_kernel"]},
+                  "bytes_per_step": int(dbytes), "gpu_launches": 2 * dsteps}
+        del dq, dk, dv, do, ws
+        torch.cuda.empty_cache()
+
+    # ---------------------------------------------------------------- other prefill workloads
+    extra = {}
+    if not args.no_extra:
+        for name in EXTRA:
+            we = synth.WORKLOADS[name]
+            f_e, c_e = prefill_flops(fattn, we)
+            eq, ek, ev = synth.make_inputs(we, device=dev, seed=we.seed + rank)
+            eo = torch.empty_like(eq)
+            el = torch.empty((we.B, we.H, we.Lq), dtype=torch.float32, device=dev)
+
+            def estep():
+                fattn.attn_fwd(eq, ek, ev, o=eo, lse=el, scale=we.scale, causal=we.causal,
+                               window_left=we.window_left, window_right=we.window_right)
+
+            esteps = max(3, min(args.steps, 10))
+            ems = timed(world, estep, esteps, 2)
+            tf = f_e / (ems * 1e-3) / 1e12
+            extra[name] = {"value": world * tf, "unit": "TFLOP/s", "ms_per_step": ems, "steps": esteps,
+                           "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
+                           "kv_tiles_visited_per_head": c_e["visited"], "kv_tiles_total_per_head": c_e["total"],
+                           "config": we.describe()}
+            del eq, ek, ev, eo, el
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_sample(w)
+
+    if rank == 0:
+        line = {"metric": "attention fwd TFLOP/s (in-mask FLOPs) & % bf16 tensor peak; decode HBM GB/s",
+                "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {**w.describe(), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                           "l2": "inputs 201 MB (Q+K+V) > 126 MB L2, no flush",
+                           "kv_tiles_visited_per_head": counts["visited"],
+                           "kv_tiles_total_per_head": counts["total"]},
+                "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
+                "clocks": clocks, "decode": decode, "extra": extra, "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

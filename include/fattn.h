@@ -1,0 +1,166 @@
+/*
+ * fattn.h -- C ABI of libfattn: exact, IO-aware tiled attention on B200 (sm_100a).
+ *
+ * What is computed.  For every batch element b, head h and query row i:
+ *
+ *     O[b,h,i,:] = sum_j softmax_j(scale * q_i . k_j) v_j        over allowed j
+ *     LSE[b,h,i] = ln sum_j exp(scale * q_i . k_j)               over allowed j
+ *
+ * the attention formula of the sliding-window FlashAttention prefill page
+ * (m.xxqk.cn/news/265020) §2, evaluated with the tiled online softmax of §3.2
+ * (running row max m, running sum l, rescale alpha = exp(m_old - m_new) of the
+ * accumulator) so the n x n score matrix never reaches device memory, and with
+ * the band mask of §4 / §4.1 evaluated by block skipping (§5.1, §5.3, §7.3):
+ * KV tiles that hold no allowed pair are never loaded or multiplied.
+ *
+ * The mask.  window_size = (window_left, window_right) as in §7.1:
+ *   key j is allowed for query i iff, with pos = i + (Lk - Lq),
+ *     j < Lk                                   (and j < seqlens_k[b] in decode)
+ *     causal == 0 || j <= pos
+ *     window_right < 0 || j <= pos + window_right
+ *     window_left  < 0 || j >= pos - window_left
+ *   A negative window means "unbounded on that side"; causal = 1 clamps the
+ *   right window to 0.  Bounds are inclusive: window_left = window_right = w
+ *   is the bidirectional band |i - j| <= w of §4.  When Lq != Lk, query i sits
+ *   at key position i + Lk - Lq (bottom-right alignment; the pages only treat
+ *   Lq == Lk).  A query row with no allowed key gets O = 0 and LSE = -inf.
+ *
+ * Layout.  Q is [B, H, Lq, d], K and V are [B, H, Lk, d], O is [B, H, Lq, d],
+ * LSE is [B, H, Lq]: dense, row-major, d innermost, no padding.  LSE is the
+ * natural-log log-sum-exp including `scale`, in fp32.
+ *
+ * Ownership and execution.  Every pointer argument named as a device pointer
+ * is device memory owned by the caller, valid until the enqueued work is done.
+ * Calls enqueue asynchronously on `stream` (a cudaStream_t, NULL = the legacy
+ * default stream) and return once enqueued; the library allocates no device
+ * memory.  Calls are thread-safe.
+ *
+ * Errors.  Every entry point returns a fattn_status; nothing aborts or throws.
+ * Argument checks run before any CUDA call, so a rejected call enqueues
+ * nothing.  A failed launch returns FATTN_ERR_CUDA.  The prefill kernel bounds
+ * every wait; if a wait runs out it records FATTN_ERR_TIMEOUT in a device
+ * status word that fattn_device_status() reads back.
+ */
+#ifndef FATTN_H
+#define FATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FATTN_OK = 0,
+    FATTN_ERR_INVALID_ARG = -1,   /* null pointer, non-positive size, bad window, scale <= 0 */
+    FATTN_ERR_UNSUPPORTED = -2,   /* head dim other than 64 / 128, or sizes beyond int32 indexing */
+    FATTN_ERR_MISALIGNED = -3,    /* a tensor base address not 16-byte aligned */
+    FATTN_ERR_WORKSPACE = -4,     /* decode workspace null or smaller than attn_decode_workspace_bytes */
+    FATTN_ERR_CUDA = -5,          /* a CUDA runtime call or launch failed */
+    FATTN_ERR_TIMEOUT = -6,       /* a bounded in-kernel wait expired (see fattn_device_status) */
+    FATTN_ERR_NO_DEVICE = -7      /* no usable sm_100 device for the current context */
+} fattn_status;
+
+/*
+ * attn_fwd -- bf16 prefill forward (tensor cores: tcgen05 MMAs into tensor
+ * memory, TMA-staged K/V tiles, warp-specialised pipeline).
+ *
+ *   q, k, v   device, bf16 [B,H,Lq,d] / [B,H,Lk,d] / [B,H,Lk,d], 16-byte aligned
+ *   o         device, bf16 [B,H,Lq,d], 16-byte aligned (written)
+ *   lse       device, fp32 [B,H,Lq] (written), or NULL to skip it
+ *   B, H, Lq, Lk >= 1;  d in {64, 128};  scale > 0 (finite), usually 1/sqrt(d)
+ *   causal, window_left, window_right: the mask above
+ *   stream    cudaStream_t
+ *
+ * Precision: products in bf16 with fp32 accumulation; the probabilities P are
+ * rounded to bf16 before the P.V product; O is rounded to bf16 (round to
+ * nearest even) after the final division by l.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int H, int Lq, int Lk, int d, float scale,
+             int causal, int window_left, int window_right, void* stream);
+
+/*
+ * attn_fwd_counted -- attn_fwd that also adds, to *kv_tiles_visited (device,
+ * unsigned 64-bit, caller-zeroed), the number of (128-row Q tile, 128-key KV
+ * tile) pairs the kernel actually loaded and multiplied.  It is the evidence
+ * that out-of-band tiles are skipped (§5.1, §9.1 "blocks computed and KV
+ * blocks visited"); the count equals attn_count_blocks(..., 128, 128) visited.
+ */
+int attn_fwd_counted(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int Lq, int Lk, int d, float scale,
+                     int causal, int window_left, int window_right,
+                     unsigned long long* kv_tiles_visited, void* stream);
+
+/*
+ * attn_fwd_f32 -- the same operation on fp32 Q/K/V/O with fp32 arithmetic on
+ * the CUDA cores (no tensor-core rounding), for exactness checks.  Arguments
+ * as attn_fwd with fp32 tensors; d in {64, 128}; lse nullable.
+ */
+int attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
+                 int B, int H, int Lq, int Lk, int d, float scale,
+                 int causal, int window_left, int window_right, void* stream);
+
+/*
+ * attn_decode_splitkv -- split-KV decode for one new query per sequence (flash
+ * decoding: "算子与编译器：FlashAttention 与长上下文" §4, short query and long
+ * K/V, parallel along the KV axis).  Split s of num_splits covers keys
+ * [s*c, min((s+1)*c, seqlens_k[b])) with c = ceil(Lk / num_splits); each
+ * split writes a normalised partial output and its LSE, and a merge kernel
+ * combines them: lse = logsumexp_s(lse_s), o = sum_s exp(lse_s - lse) o_s.
+ *
+ *   q          device, bf16 [B,H,1,d]
+ *   k_cache    device, bf16 [B,H,Lk,d]
+ *   v_cache    device, bf16 [B,H,Lk,d]
+ *   o          device, bf16 [B,H,1,d] (written)
+ *   lse        device, fp32 [B,H] (written), or NULL
+ *   seqlens_k  device, int32 [B] with 0 <= seqlens_k[b] <= Lk, or NULL (all Lk).
+ *              A sequence of length 0 gets O = 0 and LSE = -inf.
+ *   num_splits 1 .. Lk, or 0 to let the library choose
+ *   workspace  device scratch of at least attn_decode_workspace_bytes(B,H,Lk,d,S)
+ *              bytes (S = the split count used), 16-byte aligned; its contents
+ *              on entry are ignored and on return are unspecified
+ */
+int attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
+                        void* o, float* lse, const int* seqlens_k,
+                        int B, int H, int Lk, int d, float scale, int num_splits,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Split count attn_decode_splitkv uses for num_splits = 0 (host only). */
+int attn_decode_auto_splits(int B, int H, int Lk, int d);
+
+/* Bytes of workspace attn_decode_splitkv needs: B*H*S*(d+1)*4 for S splits
+ * (num_splits = 0: the automatic choice for this Lk).  0 on invalid input.
+ * Host only. */
+size_t attn_decode_workspace_bytes(int B, int H, int Lk, int d, int num_splits);
+
+/*
+ * attn_count_blocks -- host-only block accounting of the scheduler (§5.4):
+ * for block_q x block_k tiles of one head's Lq x Lk score matrix,
+ *   visited = tiles holding at least one allowed pair (exactly the tiles the
+ *             kernel loads: the closed-form per-Q-tile KV range of §7.3),
+ *   total   = ceil(Lq/block_q) * ceil(Lk/block_k),
+ *   partial = visited tiles that need the element mask of §5.2,
+ *   pairs   = allowed (query, key) pairs (4*d in-mask FLOPs each).
+ * Any output pointer may be NULL.
+ */
+int attn_count_blocks(int Lq, int Lk, int causal, int window_left, int window_right,
+                      int block_q, int block_k, long long* visited, long long* total,
+                      long long* partial, long long* pairs);
+
+/* Human-readable name of a fattn_status value. */
+const char* fattn_status_string(int status);
+
+/*
+ * fattn_device_status -- synchronises `stream`, then returns and clears the
+ * device status word of the current device (FATTN_OK, or FATTN_ERR_TIMEOUT if
+ * a bounded wait in a prefill kernel expired since the last call).  A debugging
+ * aid; it blocks the calling thread.
+ */
+int fattn_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FATTN_H */

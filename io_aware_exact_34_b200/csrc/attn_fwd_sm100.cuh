@@ -1,0 +1,476 @@
+// attn_fwd_sm100.cuh -- bf16 prefill forward on the 5th-generation tensor cores.
+//
+// The operation is the tiled online-softmax attention of the sliding-window
+// FlashAttention prefill page (m.xxqk.cn/news/265020) §3.1-§3.2: Q, K and V
+// are cut into 128-row tiles, each Q tile keeps its running row max m_i,
+// running sum l_i and accumulator acc on chip, every visited KV tile updates
+// them (m_new = max(m_i, rowmax s_ij), p_ij = exp(s_ij - m_new),
+// alpha = exp(m_i - m_new), l_i = alpha l_i + rowsum p_ij,
+// acc = alpha acc + p_ij v_j), and only O = acc / l_i reaches device memory.
+// KV tiles outside the band are never loaded (§5.1, §5.3, §7.3); tiles the
+// band crosses get the element mask before the softmax (§5.2).
+//
+// B200 mapping (one persistent CTA per SM, 384 threads):
+//   warp 0        TMA producer: Q tile pair, then a ring of K / V tiles
+//   warp 1        MMA issuer (one thread): S = Q K^T and O += P V with
+//                 tcgen05.mma, accumulators in tensor memory (TMEM)
+//   warps 4-7     softmax for Q tile 0 of the pair (one thread per row)
+//   warps 8-11    softmax for Q tile 1 of the pair
+// The two Q tiles share every K / V tile; while one softmax warpgroup turns
+// its S into P, the tensor core works on the other tile.
+//
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+// P (bf16, two per 32-bit column) overwrites the first 64 columns of its S
+// tile and feeds the P.V MMA straight from TMEM.
+//
+// Exact rescale skipping: the running max used for the exponentials is only
+// raised when a new row max exceeds it by more than kRescaleSlack (log2
+// units); otherwise p = 2^(x - m) <= 2^kRescaleSlack.  Numerator and
+// denominator use the same reference, so O = acc / l is unchanged (the page's
+// "skipped block == all -inf block" argument of §5.5 generalises to any
+// common reference), and O in TMEM is rescaled only when the reference moves.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "dev_prims.cuh"
+#include "sched.cuh"
+
+namespace fattn {
+
+constexpr float kRescaleSlack = 8.0f;
+
+template <int D>
+struct FwdTraits {
+    static constexpr int BQ = 128;                 // rows per Q tile (one per TMEM lane)
+    static constexpr int BK = 128;                 // keys per KV tile
+    static constexpr int CHUNK_BYTES = 128 * 128;  // 128 rows x 64 bf16: one 128-B swizzle column
+    static constexpr int NCHUNK = D / 64;
+    static constexpr int TILE_BYTES = 128 * D * 2;
+    static constexpr int NSTAGE = D == 128 ? 4 : 8;  // K/V ring slots
+    static constexpr int SMEM_Q_OFF = 0;
+    static constexpr int SMEM_RING_OFF = 2 * TILE_BYTES;
+    static constexpr int SMEM_BAR_OFF = SMEM_RING_OFF + NSTAGE * TILE_BYTES;
+    static constexpr int NBAR = 2 + 2 * NSTAGE + 6 + 1;
+    static constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NBAR * 8;
+    static constexpr int SMEM_BYTES = SMEM_MISC_OFF + 16 + 1024;  // + alignment slack
+    static constexpr int THREADS = 384;
+    // Register split: warpgroup 0 (producer, MMA issuer) lowers to REGS_LOW,
+    // the two softmax warpgroups raise to REGS_HIGH.  128*80 + 256*208 = 63488
+    // <= 384 threads * 168 registers = 64512, the pool the block is launched
+    // with; the host refuses to launch unless the compiled register count
+    // provides that pool.
+    static constexpr uint32_t REGS_LAUNCH = 168;
+    static constexpr uint32_t REGS_LOW = 80;
+    static constexpr uint32_t REGS_HIGH = 208;
+    static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= THREADS * REGS_LAUNCH, "register split");
+    static constexpr uint32_t TMEM_COLS = 512;
+    __host__ __device__ static constexpr uint32_t tm_s(int t) { return static_cast<uint32_t>(t) * 128u; }
+    __host__ __device__ static constexpr uint32_t tm_o(int t) { return 256u + static_cast<uint32_t>(t) * D; }
+    static_assert(D == 64 || D == 128, "head dim");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+struct FwdParams {
+    void* o;
+    float* lse;
+    unsigned long long* visited;
+    int B, H, Lq, Lk;
+    float scale_log2;  // scale * log2(e)
+    int causal, window_left, window_right;
+    int n_pairs, n_items;
+};
+
+// The two Q tiles of one work item and the KV tiles they visit.
+struct PairTiles {
+    int bh;
+    long long q_first[2], q_last[2];
+    bool exists[2];
+    int lo_t[2], hi_t[2];
+    int lo, hi;  // union range
+};
+
+__device__ __forceinline__ int snake_item(int round, int cta, int grid) {
+    // Work items are ordered longest first; alternating the direction of
+    // each round evens out the per-CTA total.
+    return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
+}
+
+__device__ __forceinline__ PairTiles pair_tiles(const FwdParams& p, const Band& band, int item) {
+    PairTiles ts;
+    const int BH = p.B * p.H;
+    const int pair = p.n_pairs - 1 - item / BH;
+    ts.bh = item % BH;
+    ts.lo = 0x7fffffff;
+    ts.hi = 0;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const long long q_first = static_cast<long long>(2 * pair + t) * 128;
+        ts.q_first[t] = q_first;
+        ts.exists[t] = q_first < p.Lq;
+        ts.q_last[t] = q_first + 127 < p.Lq - 1 ? q_first + 127 : p.Lq - 1;
+        int lo = 0, hi = 0;
+        if (ts.exists[t]) kv_tile_range(band, q_first, ts.q_last[t], 128, &lo, &hi);
+        ts.lo_t[t] = lo;
+        ts.hi_t[t] = hi;
+        if (lo < hi) {
+            ts.lo = lo < ts.lo ? lo : ts.lo;
+            ts.hi = hi > ts.hi ? hi : ts.hi;
+        }
+    }
+    if (ts.lo >= ts.hi) ts.lo = ts.hi = 0;
+    return ts;
+}
+
+// What one softmax thread needs for its query row in one work item: the KV
+// tile range of its Q tile, the key bounds of its row and the key window in
+// which a tile needs no mask at all (absolute key indices, clamped to int).
+struct RowPlan {
+    long long orow;   // row index into O / LSE ([B*H*Lq])
+    int lo, hi;       // KV tile range of the Q tile
+    int key_lo, key_hi;   // allowed keys of this row: [key_lo, key_hi]
+    int full_lo, full_hi; // a tile [k0, k0+127] is unmasked iff k0 >= full_lo && k0+127 <= full_hi
+    bool tile_exists, valid;
+};
+
+__device__ __forceinline__ int clamp_int(long long x) {
+    return static_cast<int>(x < -(1LL << 30) ? -(1LL << 30) : (x > (1LL << 30) ? (1LL << 30) : x));
+}
+
+__device__ __forceinline__ RowPlan row_plan(const FwdParams& p, int item, int t, int row) {
+    RowPlan rp;
+    const Band band = make_band(p.Lq, p.Lk, p.causal, p.window_left, p.window_right);
+    const int BH = p.B * p.H;
+    const int pair = p.n_pairs - 1 - item / BH;
+    const int bh = item % BH;
+    const long long q_first = static_cast<long long>(2 * pair + t) * 128;
+    const long long q_last = q_first + 127 < p.Lq - 1 ? q_first + 127 : p.Lq - 1;
+    const long long i = q_first + row;
+    rp.tile_exists = q_first < p.Lq;
+    rp.valid = i < p.Lq;
+    rp.orow = static_cast<long long>(bh) * p.Lq + i;
+    rp.lo = rp.hi = 0;
+    if (rp.tile_exists) kv_tile_range(band, q_first, q_last, 128, &rp.lo, &rp.hi);
+    int lo_col, hi_col;
+    row_col_bounds(band, i, 0, &lo_col, &hi_col);
+    rp.key_lo = lo_col;
+    rp.key_hi = hi_col;
+    long long fhi = band.Lk - 1;
+    if (band.right >= 0 && q_first + band.shift + band.right < fhi) fhi = q_first + band.shift + band.right;
+    const long long flo = band.left >= 0 ? q_last + band.shift - band.left : 0;
+    rp.full_lo = clamp_int(flo);
+    rp.full_hi = clamp_int(fhi);
+    return rp;
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+    using T = FwdTraits<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t sQ = base + T::SMEM_Q_OFF;
+    const uint32_t sRing = base + T::SMEM_RING_OFF;
+    const uint32_t bar0 = base + T::SMEM_BAR_OFF;
+    const uint32_t q_full = bar0;
+    const uint32_t q_empty = bar0 + 8;
+    const uint32_t kv_full0 = bar0 + 16;
+    const uint32_t kv_empty0 = kv_full0 + 8 * T::NSTAGE;
+    const uint32_t s_full0 = kv_empty0 + 8 * T::NSTAGE;
+    const uint32_t p_ready0 = s_full0 + 16;
+    const uint32_t o_full0 = p_ready0 + 16;
+    const uint32_t drain_bar = o_full0 + 16;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + T::SMEM_MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + T::SMEM_MISC_OFF + 4);
+    int* status = &g_fattn_status;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int s = 0; s < T::NSTAGE; ++s) {
+            mbar_init(kv_full0 + 8 * s, 1);
+            mbar_init(kv_empty0 + 8 * s, 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(s_full0 + 8 * t, 1);
+            mbar_init(p_ready0 + 8 * t, 128);
+            mbar_init(o_full0 + 8 * t, 1);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_map(&tm_q);
+        tma_prefetch_map(&tm_k);
+        tma_prefetch_map(&tm_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_holder), T::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+
+    if (warp < 4) {
+      warpgroup_reg_lower<T::REGS_LOW>();
+      const Band band = make_band(p.Lq, p.Lk, p.causal, p.window_left, p.window_right);
+      if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t ring = 0, q_round = 0;
+            bool ok = true;
+            for (int round = 0; ok; ++round) {
+                const int item = snake_item(round, blockIdx.x, gridDim.x);
+                if (item >= p.n_items) break;
+                const PairTiles ts = pair_tiles(p, band, item);
+                if (ts.lo >= ts.hi) continue;
+                if (q_round > 0) {
+                    ok = mbar_wait(q_empty, (q_round - 1) & 1u, abort_flag, status, -6);
+                    if (!ok) break;
+                }
+                mbar_arrive_expect_tx(q_full, 2 * T::TILE_BYTES);
+                for (int t = 0; t < 2; ++t)
+                    for (int c = 0; c < T::NCHUNK; ++c)
+                        tma_load_3d(sQ + t * T::TILE_BYTES + c * T::CHUNK_BYTES, &tm_q, q_full, c * 64,
+                                    static_cast<int>(ts.q_first[t]), ts.bh);
+                ++q_round;
+                for (int j = ts.lo; j < ts.hi && ok; ++j) {
+                    for (int kv = 0; kv < 2; ++kv) {
+                        const uint32_t slot = ring % T::NSTAGE, use = ring / T::NSTAGE;
+                        if (use > 0) {
+                            ok = mbar_wait(kv_empty0 + 8 * slot, (use - 1) & 1u, abort_flag, status, -6);
+                            if (!ok) break;
+                        }
+                        const uint32_t fb = kv_full0 + 8 * slot;
+                        mbar_arrive_expect_tx(fb, T::TILE_BYTES);
+                        for (int c = 0; c < T::NCHUNK; ++c)
+                            tma_load_3d(sRing + slot * T::TILE_BYTES + c * T::CHUNK_BYTES, kv ? &tm_v : &tm_k, fb,
+                                        c * 64, j * 128, ts.bh);
+                        ++ring;
+                    }
+                }
+            }
+            // No TMA write may still be landing in shared memory when the CTA exits.
+            if (q_round > 0) mbar_wait(q_full, (q_round - 1) & 1u, nullptr, status, -6);
+            for (uint32_t s = 0; s < T::NSTAGE; ++s) {
+                if (ring > s) {
+                    const uint32_t uses = (ring - 1 - s) / T::NSTAGE + 1;
+                    mbar_wait(kv_full0 + 8 * s, (uses - 1) & 1u, nullptr, status, -6);
+                }
+            }
+        }
+      } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+            uint32_t ring = 0, q_round = 0, p_cnt[2] = {0u, 0u};
+            bool ok = true;
+            for (int round = 0; ok; ++round) {
+                const int item = snake_item(round, blockIdx.x, gridDim.x);
+                if (item >= p.n_items) break;
+                const PairTiles ts = pair_tiles(p, band, item);
+                if (ts.lo >= ts.hi) continue;
+                ok = mbar_wait(q_full, q_round & 1u, abort_flag, status, -6);
+                if (!ok) break;
+                ++q_round;
+                tc_fence_after_sync();
+                const uint32_t ring0 = ring;
+                for (int j = ts.lo; j <= ts.hi && ok; ++j) {
+                    const bool haveK = j < ts.hi;
+                    const bool haveV = j > ts.lo;
+                    const uint32_t rK = ring0 + 2u * static_cast<uint32_t>(j - ts.lo);
+                    const uint32_t rV = rK - 1u;  // V tile of KV tile j-1
+                    if (haveK) ok = mbar_wait(kv_full0 + 8 * (rK % T::NSTAGE), (rK / T::NSTAGE) & 1u, abort_flag, status, -6);
+                    if (ok && haveV) ok = mbar_wait(kv_full0 + 8 * (rV % T::NSTAGE), (rV / T::NSTAGE) & 1u, abort_flag, status, -6);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        // O_t += P_t V_{j-1}
+                        if (haveV && j - 1 >= ts.lo_t[t] && j - 1 < ts.hi_t[t]) {
+                            ok = mbar_wait(p_ready0 + 8 * t, p_cnt[t] & 1u, abort_flag, status, -6);
+                            ++p_cnt[t];
+                            if (!ok) break;
+                            tc_fence_after_sync();
+                            const uint32_t vbase = sRing + (rV % T::NSTAGE) * T::TILE_BYTES;
+                            const uint32_t first = (j - 1 == ts.lo_t[t]) ? 1u : 0u;
+#pragma unroll
+                            for (int ks = 0; ks < 8; ++ks) {
+                                const uint64_t bdesc = sdesc_sw128(vbase + ks * 2048, T::CHUNK_BYTES, 1024);
+                                mma_bf16_ts(tmem + T::tm_o(t), tmem + T::tm_s(t) + ks * 8, bdesc, idesc_pv,
+                                            (first && ks == 0) ? 0u : 1u);
+                            }
+                            if (j - 1 == ts.hi_t[t] - 1) mma_commit(o_full0 + 8 * t);
+                        }
+                        // S_t = Q_t K_j^T
+                        if (haveK && j >= ts.lo_t[t] && j < ts.hi_t[t]) {
+                            const uint32_t kbase = sRing + (rK % T::NSTAGE) * T::TILE_BYTES;
+                            const uint32_t qbase = sQ + t * T::TILE_BYTES;
+#pragma unroll
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint32_t off = (ks / 4) * T::CHUNK_BYTES + (ks % 4) * 32;
+                                mma_bf16_ss(tmem + T::tm_s(t), sdesc_sw128(qbase + off, 16, 1024),
+                                            sdesc_sw128(kbase + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+                            }
+                            mma_commit(s_full0 + 8 * t);
+                        }
+                    }
+                    if (!ok) break;
+                    if (haveV) mma_commit(kv_empty0 + 8 * (rV % T::NSTAGE));
+                    if (haveK) {
+                        mma_commit(kv_empty0 + 8 * (rK % T::NSTAGE));
+                        if (j == ts.hi - 1) mma_commit(q_empty);
+                    }
+                }
+                ring = ring0 + 2u * static_cast<uint32_t>(ts.hi - ts.lo);
+            }
+        }
+      }
+    } else {
+        // ------------------------------------------------------------ softmax warpgroups
+        warpgroup_reg_raise<T::REGS_HIGH>();
+        const int t = (warp - 4) >> 2;
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t taddr_s = tmem + lane_off + T::tm_s(t);
+        const uint32_t taddr_o = tmem + lane_off + T::tm_o(t);
+        const uint32_t s_full = s_full0 + 8 * t, p_ready = p_ready0 + 8 * t, o_full = o_full0 + 8 * t;
+        const float c_log2 = p.scale_log2;
+        uint32_t s_phase = 0, o_phase = 0;
+        bool ok = true;
+        for (int round = 0; ok; ++round) {
+            const int item = snake_item(round, blockIdx.x, gridDim.x);
+            if (item >= p.n_items) break;
+            const RowPlan rp = row_plan(p, item, t, row);
+            if (!rp.tile_exists) continue;
+            if (rp.lo >= rp.hi) {
+                // no allowed key for any row of this tile
+                if (rp.valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + rp.orow * D);
+#pragma unroll
+                    for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+                    if (p.lse) p.lse[rp.orow] = -CUDART_INF_F;
+                }
+                continue;
+            }
+            float m_used = -CUDART_INF_F, l = 0.f;
+            for (int j = rp.lo; j < rp.hi; ++j) {
+                ok = mbar_wait(s_full, s_phase & 1u, abort_flag, status, -6);
+                ++s_phase;
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after_sync();
+                uint32_t sr[4][32];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(taddr_s + q4 * 32, sr[q4]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) reg_fence(sr[q4]);
+                const int k0 = j * 128;
+                if (!(k0 >= rp.full_lo && k0 + 127 <= rp.full_hi)) {
+                    // §5.2: the boundary mask goes on before the softmax
+                    const int lo_col = rp.key_lo - k0, hi_col = rp.key_hi - k0;
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (c < lo_col || c > hi_col) sr[c >> 5][c & 31] = __float_as_uint(-CUDART_INF_F);
+                }
+                float mx = -CUDART_INF_F;
+#pragma unroll
+                for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c >> 5][c & 31]));
+                const float mx_s = mx * c_log2;
+                float alpha = 1.f;
+                bool resc = false;
+                if (mx_s > m_used + kRescaleSlack) {
+                    alpha = fast_exp2(m_used - mx_s);  // 0 when m_used is -inf
+                    resc = (j > rp.lo) && (m_used != -CUDART_INF_F);
+                    m_used = mx_s;
+                    l *= alpha;
+                }
+                const float m_safe = (m_used == -CUDART_INF_F) ? 0.f : m_used;
+                float rowsum = 0.f;
+                uint32_t pk[2][32];
+#pragma unroll
+                for (int c = 0; c < 128; c += 2) {
+                    const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c >> 5][c & 31]), c_log2, -m_safe));
+                    const float p1 = fast_exp2(fmaf(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]), c_log2, -m_safe));
+                    rowsum += p0 + p1;
+                    pk[c >> 6][(c & 63) >> 1] = pack_bf16x2(p0, p1);
+                }
+                l += rowsum;
+                tmem_st32(taddr_s, pk[0]);
+                tmem_st32(taddr_s + 32, pk[1]);
+                if (__any_sync(0xffffffffu, resc)) {
+                    const float a = resc ? alpha : 1.f;
+#pragma unroll 1
+                    for (int ch = 0; ch < D / 32; ++ch) {
+                        uint32_t orr[32];
+                        tmem_ld32(taddr_o + ch * 32, orr);
+                        tmem_wait_ld();
+                        reg_fence(orr);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * a);
+                        tmem_st32(taddr_o + ch * 32, orr);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before_sync();
+                mbar_arrive(p_ready);
+            }
+            if (!ok) break;
+            // epilogue: O = acc / l, LSE = (m + log2 l) ln 2
+            ok = mbar_wait(o_full, o_phase & 1u, abort_flag, status, -6);
+            ++o_phase;
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after_sync();
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + rp.orow * D;
+#pragma unroll 1
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t orr[32];
+                tmem_ld32(taddr_o + ch * 32, orr);
+                tmem_wait_ld();
+                reg_fence(orr);
+                if (rp.valid) {
+                    uint32_t pk16[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pk16[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l, __uint_as_float(orr[2 * e + 1]) * inv_l);
+                    uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk16[4 * v], pk16[4 * v + 1], pk16[4 * v + 2], pk16[4 * v + 3]);
+                }
+            }
+            if (rp.valid && p.lse) p.lse[rp.orow] = l > 0.f ? (m_used + __log2f(l)) * 0.6931471805599453f : -CUDART_INF_F;
+            if (p.visited && quarter == 0 && lane == 0)
+                atomicAdd(p.visited, static_cast<unsigned long long>(rp.hi - rp.lo));
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        if (lane == 0) {
+            // every MMA this CTA issued has finished before TMEM is released
+            mma_commit(drain_bar);
+            mbar_wait(drain_bar, 0, nullptr, status, -6);
+        }
+        __syncwarp();
+        tmem_dealloc(tmem, T::TMEM_COLS);
+    }
+}
+
+}  // namespace fattn

@@ -1,0 +1,323 @@
+// fattn_api.cu -- the C ABI of libfattn (declared in include/fattn.h).
+//
+// One translation unit: argument checks (before any CUDA call), TMA tensor
+// map encoding, per-device launch attributes, kernel launches, host-side block
+// accounting and the device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "fattn.h"
+
+#include "attn_fwd_f32.cuh"
+#include "attn_fwd_sm100.cuh"
+#include "decode_splitkv.cuh"
+#include "sched.cuh"
+
+namespace {
+
+using namespace fattn;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    bool sm100 = false;
+    bool fwd_regs_ok = false;  // the prefill kernels' register pool covers their split
+    int num_sms = 0;
+};
+
+// The prefill kernel's warpgroups change their register budgets with
+// setmaxnreg; the sum must fit the pool the block is launched with, or the
+// raising warpgroups would wait forever.  Checked against the compiled kernel.
+template <int D>
+bool fwd_register_pool_ok() {
+    cudaFuncAttributes a;
+    if (cudaFuncGetAttributes(&a, attn_fwd_sm100_kernel<D>) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    using T = FwdTraits<D>;
+    return static_cast<long long>(a.numRegs) * T::THREADS >=
+           128LL * T::REGS_LOW + 256LL * T::REGS_HIGH;
+}
+
+std::mutex g_mutex;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Current device, checked to be sm_100 with the kernels' launch attributes set.
+int device_ready(DeviceInfo* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return FATTN_ERR_NO_DEVICE;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return FATTN_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo& di = g_dev[dev];
+    if (!di.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return FATTN_ERR_NO_DEVICE;
+        }
+        di.sm100 = (major == 10 && minor == 0);
+        di.num_sms = sms;
+        if (di.sm100) {
+            cudaError_t e = cudaSuccess;
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128>::SMEM_BYTES);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64>::SMEM_BYTES);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, F32Traits<128>::SMEM_BYTES);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, F32Traits<64>::SMEM_BYTES);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return FATTN_ERR_CUDA;
+            }
+            di.fwd_regs_ok = fwd_register_pool_ok<128>() && fwd_register_pool_ok<64>();
+            if (g_encode == nullptr) {
+                void* fn = nullptr;
+                cudaDriverEntryPointQueryResult q;
+                if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                    q != cudaDriverEntryPointSuccess || fn == nullptr) {
+                    cudaGetLastError();
+                    return FATTN_ERR_CUDA;
+                }
+                g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+            }
+        }
+        di.ready = true;
+    }
+    if (!di.sm100) return FATTN_ERR_NO_DEVICE;
+    *out = di;
+    return FATTN_OK;
+}
+
+// Common checks of the prefill entry points (host only, no CUDA call).
+int check_prefill(const void* q, const void* k, const void* v, const void* o, const void* lse, int B, int H,
+                  int Lq, int Lk, int d, float scale) {
+    if (!q || !k || !v || !o) return FATTN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || Lq < 1 || Lk < 1) return FATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return FATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FATTN_ERR_UNSUPPORTED;
+    const long long bh = static_cast<long long>(B) * H;
+    if (bh > 0x7fffffffLL || Lq > 0x7fffff00 || Lk > 0x7fffff00) return FATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FATTN_ERR_MISALIGNED;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FATTN_ERR_MISALIGNED;
+    return FATTN_OK;
+}
+
+// [B*H, L, d] bf16 tensor, 64-element x 128-row boxes, 128-byte swizzle.
+int encode_map(CUtensorMap* map, const void* base, int d, long long L, long long BH) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(L) * d * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FATTN_OK : FATTN_ERR_CUDA;
+}
+
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq, int Lk, int d,
+               float scale, int causal, int wl, int wr, unsigned long long* visited, void* stream) {
+    int st = check_prefill(q, k, v, o, lse, B, H, Lq, Lk, d, scale);
+    if (st != FATTN_OK) return st;
+    DeviceInfo di;
+    st = device_ready(&di);
+    if (st != FATTN_OK) return st;
+    if (!di.fwd_regs_ok) return FATTN_ERR_UNSUPPORTED;
+    const long long BH = static_cast<long long>(B) * H;
+    const long long n_qtiles = (Lq + 127) / 128;
+    const long long n_pairs = (n_qtiles + 1) / 2;
+    const long long n_items = BH * n_pairs;
+    if (n_items > 0x7fffffffLL) return FATTN_ERR_UNSUPPORTED;
+    CUtensorMap mq, mk, mv;
+    if (encode_map(&mq, q, d, Lq, BH) != FATTN_OK || encode_map(&mk, k, d, Lk, BH) != FATTN_OK ||
+        encode_map(&mv, v, d, Lk, BH) != FATTN_OK)
+        return FATTN_ERR_CUDA;
+    FwdParams p;
+    p.o = o;
+    p.lse = lse;
+    p.visited = visited;
+    p.B = B;
+    p.H = H;
+    p.Lq = Lq;
+    p.Lk = Lk;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.window_left = wl < 0 ? -1 : wl;
+    p.window_right = wr < 0 ? -1 : wr;
+    p.n_pairs = static_cast<int>(n_pairs);
+    p.n_items = static_cast<int>(n_items);
+    const int grid = static_cast<int>(n_items < di.num_sms ? n_items : di.num_sms);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (d == 128)
+        attn_fwd_sm100_kernel<128><<<grid, FwdTraits<128>::THREADS, FwdTraits<128>::SMEM_BYTES, s>>>(mq, mk, mv, p);
+    else
+        attn_fwd_sm100_kernel<64><<<grid, FwdTraits<64>::THREADS, FwdTraits<64>::SMEM_BYTES, s>>>(mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? FATTN_OK : FATTN_ERR_CUDA;
+}
+
+int auto_splits(int B, int H, int Lk) {
+    (void)B;
+    (void)H;
+    // largest power of two <= 64 that still leaves at least 1024 keys per split
+    int S = 1;
+    while (S < 64 && static_cast<long long>(Lk) / (S * 2) >= 1024) S *= 2;
+    return S;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq, int Lk, int d,
+             float scale, int causal, int window_left, int window_right, void* stream) {
+    return launch_fwd(q, k, v, o, lse, B, H, Lq, Lk, d, scale, causal, window_left, window_right, nullptr, stream);
+}
+
+int attn_fwd_counted(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq, int Lk,
+                     int d, float scale, int causal, int window_left, int window_right,
+                     unsigned long long* kv_tiles_visited, void* stream) {
+    if (!kv_tiles_visited) return FATTN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(kv_tiles_visited) & 7u) return FATTN_ERR_MISALIGNED;
+    return launch_fwd(q, k, v, o, lse, B, H, Lq, Lk, d, scale, causal, window_left, window_right, kv_tiles_visited,
+                      stream);
+}
+
+int attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int Lq, int Lk,
+                 int d, float scale, int causal, int window_left, int window_right, void* stream) {
+    int st = check_prefill(q, k, v, o, lse, B, H, Lq, Lk, d, scale);
+    if (st != FATTN_OK) return st;
+    if (static_cast<long long>(B) * H > 65535) return FATTN_ERR_UNSUPPORTED;  // grid.y
+    DeviceInfo di;
+    st = device_ready(&di);
+    if (st != FATTN_OK) return st;
+    const int wl = window_left < 0 ? -1 : window_left;
+    const int wr = window_right < 0 ? -1 : window_right;
+    dim3 grid((Lq + 31) / 32, B * H);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (d == 128)
+        attn_fwd_f32_kernel<128><<<grid, 128, F32Traits<128>::SMEM_BYTES, s>>>(q, k, v, o, lse, Lq, Lk, scale,
+                                                                              causal ? 1 : 0, wl, wr);
+    else
+        attn_fwd_f32_kernel<64><<<grid, 128, F32Traits<64>::SMEM_BYTES, s>>>(q, k, v, o, lse, Lq, Lk, scale,
+                                                                            causal ? 1 : 0, wl, wr);
+    return cudaGetLastError() == cudaSuccess ? FATTN_OK : FATTN_ERR_CUDA;
+}
+
+int attn_decode_auto_splits(int B, int H, int Lk, int d) {
+    if (B < 1 || H < 1 || Lk < 1 || (d != 64 && d != 128)) return FATTN_ERR_INVALID_ARG;
+    return auto_splits(B, H, Lk);
+}
+
+size_t attn_decode_workspace_bytes(int B, int H, int Lk, int d, int num_splits) {
+    if (B < 1 || H < 1 || Lk < 1 || d < 1 || num_splits < 0) return 0;
+    const long long S = num_splits == 0 ? auto_splits(B, H, Lk) : num_splits;
+    return static_cast<size_t>(B) * H * S * (static_cast<size_t>(d) + 1) * sizeof(float);
+}
+
+int attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                        const int* seqlens_k, int B, int H, int Lk, int d, float scale, int num_splits,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    if (!q || !k_cache || !v_cache || !o) return FATTN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || Lk < 1 || num_splits < 0) return FATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return FATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FATTN_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 65535 || Lk > 0x7fffff00) return FATTN_ERR_UNSUPPORTED;
+    const int S = num_splits == 0 ? auto_splits(B, H, Lk) : num_splits;
+    if (S > Lk || S > 0x7fffffff / 1) return FATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return FATTN_ERR_MISALIGNED;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FATTN_ERR_MISALIGNED;
+    if (seqlens_k && (reinterpret_cast<uintptr_t>(seqlens_k) & 3u)) return FATTN_ERR_MISALIGNED;
+    const size_t need = attn_decode_workspace_bytes(B, H, Lk, d, S);
+    if (!workspace || workspace_bytes < need) return FATTN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FATTN_ERR_MISALIGNED;
+    DeviceInfo di;
+    int st = device_ready(&di);
+    if (st != FATTN_OK) return st;
+    float* ws_o = static_cast<float*>(workspace);
+    float* ws_lse = ws_o + static_cast<size_t>(B) * H * S * d;
+    const int chunk = static_cast<int>((static_cast<long long>(Lk) + S - 1) / S);
+    const float c_log2 = scale * 1.4426950408889634f;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    dim3 grid(S, H, B);
+    const auto* qb = static_cast<const __nv_bfloat16*>(q);
+    const auto* kb = static_cast<const __nv_bfloat16*>(k_cache);
+    const auto* vb = static_cast<const __nv_bfloat16*>(v_cache);
+    auto* ob = static_cast<__nv_bfloat16*>(o);
+    if (d == 128) {
+        decode_split_kernel<128><<<grid, 256, 0, s>>>(qb, kb, vb, seqlens_k, ws_o, ws_lse, H, Lk, S, chunk, c_log2);
+        decode_merge_kernel<128><<<B * H, 128, 0, s>>>(ws_o, ws_lse, ob, lse, S);
+    } else {
+        decode_split_kernel<64><<<grid, 256, 0, s>>>(qb, kb, vb, seqlens_k, ws_o, ws_lse, H, Lk, S, chunk, c_log2);
+        decode_merge_kernel<64><<<B * H, 64, 0, s>>>(ws_o, ws_lse, ob, lse, S);
+    }
+    return cudaGetLastError() == cudaSuccess ? FATTN_OK : FATTN_ERR_CUDA;
+}
+
+int attn_count_blocks(int Lq, int Lk, int causal, int window_left, int window_right, int block_q, int block_k,
+                      long long* visited, long long* total, long long* partial, long long* pairs) {
+    if (Lq < 1 || Lk < 1 || block_q < 1 || block_k < 1) return FATTN_ERR_INVALID_ARG;
+    const Band band = make_band(Lq, Lk, causal, window_left, window_right);
+    const long long nq = (Lq + block_q - 1) / block_q, nk = (Lk + block_k - 1) / block_k;
+    long long n_visited = 0, n_partial = 0, n_pairs = 0;
+    for (long long t = 0; t < nq; ++t) {
+        const long long q_first = t * block_q;
+        const long long q_last = q_first + block_q - 1 < Lq - 1 ? q_first + block_q - 1 : Lq - 1;
+        int lo = 0, hi = 0;
+        kv_tile_range(band, q_first, q_last, block_k, &lo, &hi);
+        n_visited += hi - lo;
+        for (int j = lo; j < hi; ++j)
+            if (!tile_is_full(band, q_first, q_last, static_cast<long long>(j) * block_k, block_k)) ++n_partial;
+    }
+    for (long long i = 0; i < Lq; ++i) {
+        int lo_col = 0, hi_col = 0;
+        row_col_bounds(band, i, 0, &lo_col, &hi_col);
+        if (hi_col >= lo_col) n_pairs += static_cast<long long>(hi_col) - lo_col + 1;
+    }
+    if (visited) *visited = n_visited;
+    if (total) *total = nq * nk;
+    if (partial) *partial = n_partial;
+    if (pairs) *pairs = n_pairs;
+    return FATTN_OK;
+}
+
+const char* fattn_status_string(int status) {
+    switch (status) {
+        case FATTN_OK: return "FATTN_OK";
+        case FATTN_ERR_INVALID_ARG: return "FATTN_ERR_INVALID_ARG: invalid argument";
+        case FATTN_ERR_UNSUPPORTED: return "FATTN_ERR_UNSUPPORTED: unsupported head dim or size";
+        case FATTN_ERR_MISALIGNED: return "FATTN_ERR_MISALIGNED: pointer not 16-byte aligned";
+        case FATTN_ERR_WORKSPACE: return "FATTN_ERR_WORKSPACE: workspace missing or too small";
+        case FATTN_ERR_CUDA: return "FATTN_ERR_CUDA: CUDA call or launch failed";
+        case FATTN_ERR_TIMEOUT: return "FATTN_ERR_TIMEOUT: a bounded in-kernel wait expired";
+        case FATTN_ERR_NO_DEVICE: return "FATTN_ERR_NO_DEVICE: no usable sm_100 device";
+        default: return "unknown fattn status";
+    }
+}
+
+int fattn_device_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return FATTN_ERR_CUDA;
+    }
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, fattn::g_fattn_status, sizeof(int)) != cudaSuccess ||
+        cudaMemcpyToSymbol(fattn::g_fattn_status, &zero, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return FATTN_ERR_CUDA;
+    }
+    return v;
+}
+
+}  // extern "C"

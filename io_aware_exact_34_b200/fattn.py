@@ -1,0 +1,180 @@
+"""Python binding of libfattn: argument marshalling over the C ABI only.
+
+Every function here takes torch tensors, checks their dtype / device / layout,
+passes raw pointers, sizes and the current CUDA stream to the library of the
+same name, and raises ``FattnError`` on a non-zero status.  All arithmetic runs
+in the library's CUDA kernels; there is no fallback of any kind.  If the
+shared library is missing, importing this module fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfattn.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libfattn.so is not built ({_LIB_PATH}); run "
+                      "`python -m io_aware_exact_34_b200.build`")
+lib = ctypes.CDLL(_LIB_PATH)
+
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_llp = ctypes.POINTER(ctypes.c_longlong)
+lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp]
+lib.attn_fwd.restype = _i
+lib.attn_fwd_counted.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp, _vp]
+lib.attn_fwd_counted.restype = _i
+lib.attn_fwd_f32.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp]
+lib.attn_fwd_f32.restype = _i
+lib.attn_decode_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz, _vp]
+lib.attn_decode_splitkv.restype = _i
+lib.attn_decode_auto_splits.argtypes = [_i, _i, _i, _i]
+lib.attn_decode_auto_splits.restype = _i
+lib.attn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+lib.attn_decode_workspace_bytes.restype = _sz
+lib.attn_count_blocks.argtypes = [_i, _i, _i, _i, _i, _i, _i, _llp, _llp, _llp, _llp]
+lib.attn_count_blocks.restype = _i
+lib.fattn_status_string.argtypes = [_i]
+lib.fattn_status_string.restype = ctypes.c_char_p
+lib.fattn_device_status.argtypes = [_vp]
+lib.fattn_device_status.restype = _i
+
+FATTN_OK = 0
+FATTN_ERR_INVALID_ARG = -1
+FATTN_ERR_UNSUPPORTED = -2
+FATTN_ERR_MISALIGNED = -3
+FATTN_ERR_WORKSPACE = -4
+FATTN_ERR_CUDA = -5
+FATTN_ERR_TIMEOUT = -6
+FATTN_ERR_NO_DEVICE = -7
+
+
+class FattnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib.fattn_status_string(status).decode()}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != FATTN_OK:
+        raise FattnError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _want(t, dtype, ndim, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype or t.dim() != ndim or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous {dtype} CUDA tensor with {ndim} dims, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, window_left=-1, window_right=-1,
+             need_lse=True):
+    """bf16 prefill forward.  q: [B,H,Lq,d], k, v: [B,H,Lk,d] -> (o, lse)."""
+    _want(q, torch.bfloat16, 4, "q")
+    _want(k, torch.bfloat16, 4, "k")
+    _want(v, torch.bfloat16, 4, "v")
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and need_lse:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    _check(lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Lq, Lk, d, scale,
+                        int(bool(causal)), int(window_left), int(window_right), _stream()), "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_counted(q, k, v, counter, o=None, lse=None, scale=None, causal=False, window_left=-1,
+                     window_right=-1):
+    """attn_fwd that adds the number of KV tiles visited to ``counter``
+    (a zeroed uint64/int64 CUDA tensor with one element)."""
+    _want(q, torch.bfloat16, 4, "q")
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    _check(lib.attn_fwd_counted(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Lq, Lk, d, scale,
+                                int(bool(causal)), int(window_left), int(window_right), _ptr(counter),
+                                _stream()), "attn_fwd_counted")
+    return o, lse
+
+
+def attn_fwd_f32(q, k, v, o=None, lse=None, scale=None, causal=False, window_left=-1, window_right=-1):
+    """fp32 prefill forward on the CUDA cores.  Same arguments as attn_fwd."""
+    _want(q, torch.float32, 4, "q")
+    _want(k, torch.float32, 4, "k")
+    _want(v, torch.float32, 4, "v")
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    _check(lib.attn_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Lq, Lk, d, scale,
+                            int(bool(causal)), int(window_left), int(window_right), _stream()), "attn_fwd_f32")
+    return o, lse
+
+
+def attn_decode_auto_splits(B, H, Lk, d) -> int:
+    return lib.attn_decode_auto_splits(B, H, Lk, d)
+
+
+def attn_decode_workspace_bytes(B, H, Lk, d, num_splits=0) -> int:
+    return lib.attn_decode_workspace_bytes(B, H, Lk, d, num_splits)
+
+
+def attn_decode_splitkv(q, k_cache, v_cache, o=None, lse=None, seqlens_k=None, scale=None,
+                        num_splits=0, workspace=None):
+    """Split-KV decode.  q: [B,H,1,d], caches [B,H,Lk,d] -> (o [B,H,1,d], lse [B,H])."""
+    _want(q, torch.bfloat16, 4, "q")
+    _want(k_cache, torch.bfloat16, 4, "k_cache")
+    _want(v_cache, torch.bfloat16, 4, "v_cache")
+    B, H, _, d = q.shape
+    Lk = k_cache.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if seqlens_k is not None:
+        _want(seqlens_k, torch.int32, 1, "seqlens_k")
+    S = num_splits if num_splits > 0 else attn_decode_auto_splits(B, H, Lk, d)
+    need = attn_decode_workspace_bytes(B, H, Lk, d, S)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    _check(lib.attn_decode_splitkv(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
+                                   _ptr(seqlens_k), B, H, Lk, d, scale, S, _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream()),
+           "attn_decode_splitkv")
+    return o, lse
+
+
+def attn_count_blocks(Lq, Lk, causal=False, window_left=-1, window_right=-1, block_q=128, block_k=128):
+    """Host-side block accounting -> dict(visited, total, partial, pairs)."""
+    out = [ctypes.c_longlong(0) for _ in range(4)]
+    _check(lib.attn_count_blocks(Lq, Lk, int(bool(causal)), window_left, window_right, block_q, block_k,
+                                 *[ctypes.byref(x) for x in out]), "attn_count_blocks")
+    return dict(visited=out[0].value, total=out[1].value, partial=out[2].value, pairs=out[3].value)
+
+
+def fattn_device_status() -> int:
+    return lib.fattn_device_status(_stream())
+
+
+def status_string(status: int) -> str:
+    return lib.fattn_status_string(status).decode()

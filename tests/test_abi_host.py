@@ -1,0 +1,150 @@
+"""Host-side tests of the C ABI: the library loads without a GPU, exports
+every function ``include/fattn.h`` declares, rejects bad arguments before any
+CUDA call, and its tile scheduler matches brute-force mask enumeration."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def fl():
+    from io_aware_exact_34_b200 import build
+    build.build()
+    from io_aware_exact_34_b200 import fattn
+    return fattn
+
+
+def _declared_functions():
+    with open(os.path.join(ROOT, "include", "fattn.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_\s\*]*?\b([A-Za-z_][A-Za-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("defined",)))
+
+
+def test_header_symbols_are_exported(fl):
+    names = _declared_functions()
+    assert {"attn_fwd", "attn_fwd_f32", "attn_decode_splitkv", "attn_count_blocks"} <= set(names)
+    lib = ctypes.CDLL(fl._LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in fattn.h but not exported"
+
+
+def test_status_strings(fl):
+    for code in range(-7, 1):
+        assert fl.status_string(code).startswith("FATTN_")
+    assert "unknown" in fl.status_string(123)
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails validation first
+
+
+def _fwd(fl, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, H=1, Lq=8, Lk=8, d=128, scale=0.1,
+         causal=0, wl=-1, wr=-1, fn="attn_fwd"):
+    return getattr(fl.lib, fn)(q, k, v, o, lse, B, H, Lq, Lk, d, scale, causal, wl, wr, None)
+
+
+@pytest.mark.parametrize("fn", ["attn_fwd", "attn_fwd_f32"])
+def test_prefill_argument_checks(fl, fn):
+    assert _fwd(fl, q=None, fn=fn) == fl.FATTN_ERR_INVALID_ARG
+    assert _fwd(fl, o=None, fn=fn) == fl.FATTN_ERR_INVALID_ARG
+    assert _fwd(fl, B=0, fn=fn) == fl.FATTN_ERR_INVALID_ARG
+    assert _fwd(fl, Lq=0, fn=fn) == fl.FATTN_ERR_INVALID_ARG
+    assert _fwd(fl, Lk=-3, fn=fn) == fl.FATTN_ERR_INVALID_ARG
+    assert _fwd(fl, scale=0.0, fn=fn) == fl.FATTN_ERR_INVALID_ARG
+    assert _fwd(fl, scale=-1.0, fn=fn) == fl.FATTN_ERR_INVALID_ARG
+    assert _fwd(fl, scale=float("inf"), fn=fn) == fl.FATTN_ERR_INVALID_ARG
+    assert _fwd(fl, scale=float("nan"), fn=fn) == fl.FATTN_ERR_INVALID_ARG
+    assert _fwd(fl, d=96, fn=fn) == fl.FATTN_ERR_UNSUPPORTED
+    assert _fwd(fl, d=256, fn=fn) == fl.FATTN_ERR_UNSUPPORTED
+    assert _fwd(fl, q=FAKE + 8, fn=fn) == fl.FATTN_ERR_MISALIGNED
+    assert _fwd(fl, o=FAKE + 2, fn=fn) == fl.FATTN_ERR_MISALIGNED
+    assert _fwd(fl, lse=FAKE + 2, fn=fn) == fl.FATTN_ERR_MISALIGNED
+
+
+def test_counted_needs_counter(fl):
+    r = fl.lib.attn_fwd_counted(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 8, 8, 128, 0.1, 0, -1, -1, None, None)
+    assert r == fl.FATTN_ERR_INVALID_ARG
+    r = fl.lib.attn_fwd_counted(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 8, 8, 128, 0.1, 0, -1, -1, FAKE + 4, None)
+    assert r == fl.FATTN_ERR_MISALIGNED
+
+
+def _dec(fl, q=FAKE, k=FAKE, v=FAKE, o=FAKE, B=2, H=2, Lk=64, d=128, S=4, ws=FAKE, ws_bytes=1 << 20,
+         scale=0.1, seqlens=None):
+    return fl.lib.attn_decode_splitkv(q, k, v, o, None, seqlens, B, H, Lk, d, scale, S, ws, ws_bytes, None)
+
+
+def test_decode_argument_checks(fl):
+    need = fl.attn_decode_workspace_bytes(2, 2, 64, 128, 4)
+    assert need == 2 * 2 * 4 * 129 * 4
+    assert _dec(fl, k=None) == fl.FATTN_ERR_INVALID_ARG
+    assert _dec(fl, S=-1) == fl.FATTN_ERR_INVALID_ARG
+    assert _dec(fl, S=65) == fl.FATTN_ERR_INVALID_ARG            # more splits than keys
+    assert _dec(fl, d=80) == fl.FATTN_ERR_UNSUPPORTED
+    assert _dec(fl, v=FAKE + 4) == fl.FATTN_ERR_MISALIGNED
+    assert _dec(fl, seqlens=FAKE + 2) == fl.FATTN_ERR_MISALIGNED
+    assert _dec(fl, ws=None) == fl.FATTN_ERR_WORKSPACE
+    assert _dec(fl, ws_bytes=need - 1) == fl.FATTN_ERR_WORKSPACE
+    assert _dec(fl, ws=FAKE + 4, ws_bytes=need) == fl.FATTN_ERR_MISALIGNED
+    assert fl.attn_decode_workspace_bytes(0, 1, 1, 128, 1) == 0
+
+
+def test_auto_splits(fl):
+    assert fl.attn_decode_auto_splits(64, 32, 32768, 128) == 32
+    assert fl.attn_decode_auto_splits(1, 1, 100, 128) == 1
+    assert fl.attn_decode_auto_splits(1, 1, 1 << 20, 64) == 64
+    assert fl.attn_decode_workspace_bytes(64, 32, 32768, 128, 0) == 64 * 32 * 32 * 129 * 4
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
+def test_valid_call_without_gpu_reports_no_device(fl):
+    assert _fwd(fl) == fl.FATTN_ERR_NO_DEVICE
+    assert _fwd(fl, fn="attn_fwd_f32", d=64) == fl.FATTN_ERR_NO_DEVICE
+    need = fl.attn_decode_workspace_bytes(2, 2, 64, 128, 4)
+    assert _dec(fl, ws_bytes=need) == fl.FATTN_ERR_NO_DEVICE
+
+
+SCHED_CASES = [
+    # (Lq, Lk, causal, wl, wr, bq, bk)
+    (4096, 4096, True, -1, -1, 128, 128),
+    (300, 300, True, -1, -1, 128, 128),
+    (1000, 1000, False, 100, 100, 128, 128),
+    (1000, 1000, True, 257, 0, 128, 128),
+    (777, 777, False, 0, 0, 128, 128),
+    (640, 640, False, 130, 7, 128, 128),
+    (129, 300, True, -1, -1, 128, 128),    # Lq < Lk (bottom-right)
+    (300, 129, True, -1, -1, 128, 128),    # Lq > Lk: leading rows without keys
+    (300, 129, False, 5, 3, 128, 128),
+    (1, 1000, False, -1, -1, 128, 128),
+    (1000, 1, True, -1, -1, 128, 128),
+    (256, 256, False, -1, -1, 64, 64),
+    (257, 333, True, 40, 0, 32, 64),
+    (513, 513, False, 64, 64, 64, 128),
+]
+
+
+@pytest.mark.parametrize("Lq,Lk,causal,wl,wr,bq,bk", SCHED_CASES)
+def test_scheduler_matches_bruteforce(fl, oracle, Lq, Lk, causal, wl, wr, bq, bk):
+    """The library's closed-form KV tile ranges (§5.4, §7.3) visit exactly the
+    tiles that hold an allowed pair; partial tiles and pair counts agree with
+    the oracle's brute-force enumeration."""
+    got = fl.attn_count_blocks(Lq, Lk, causal, wl, wr, bq, bk)
+    want = oracle.count_blocks(Lq, Lk, causal, wl, wr, bq, bk)
+    assert got == want
+
+
+def test_scheduler_page_example(fl):
+    """n = 32768, w = 2048, B = 128 (sliding-window page §5.4): 8176 of 65536."""
+    c = fl.attn_count_blocks(32768, 32768, False, 2048, 2048, 128, 128)
+    assert (c["visited"], c["total"], c["partial"]) == (8176, 65536, 480)
+    c = fl.attn_count_blocks(32768, 32768, True, 4096, 0, 128, 128)
+    assert (c["visited"], c["partial"]) == (7920, 480)
+    c = fl.attn_count_blocks(4096, 4096, True, -1, -1, 128, 128)
+    assert (c["visited"], c["partial"]) == (528, 32)
+    c = fl.attn_count_blocks(65536, 65536, True, -1, -1, 128, 128)
+    assert (c["visited"], c["partial"]) == (131328, 512)
