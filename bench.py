@@ -382,6 +382,8 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-headline", action="store_true", help="skip the headline prefill (profiling runs)")
+    ap.add_argument("--decode-batch", type=int, default=0, help="override the decode batch (profiling runs)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

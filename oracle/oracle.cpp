@@ -17,8 +17,7 @@
  *   [P1] "算子与编译器：FlashAttention 与长上下文" (charles2530.github.io)
  *        §4 (flash decoding: short query, long K/V, parallel over the KV axis)
  *
- * Readings where the pages are silent or garbled (each is listed with its
- * reason in the design notes of the repository):
+ * Readings where the pages are silent or garbled:
  *   R1  a window w is inclusive: |i - j| <= w is in band.
  *   R3  when Lq != Lk, query i sits at key position i + (Lk - Lq).
  *   R4  LSE is the natural-log log-sum-exp of the scaled scores of the row.
