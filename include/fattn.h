@@ -159,6 +159,41 @@ const char* fattn_status_string(int status);
  */
 int fattn_device_status(void* stream);
 
+/*
+ * attn_decode_splitkv_noalloc -- attn_decode_splitkv for callers that cannot
+ * allocate device memory.  The pages have no counterpart to this entry point;
+ * it exists for the library's users, not for the method.
+ *
+ * Who needs it: code that is handed only its input and output buffers, such
+ * as a plugin inside a host application or runtime that owns every device
+ * allocation, or a service that runs under a fixed memory budget and must not
+ * let a request fail on a workspace allocation; cudaMalloc / cudaFree can also
+ * block or synchronise the device, which such callers must avoid.  Those
+ * callers still pass q, the caches, o and lse; the split partials go to a
+ * scratch array compiled into this library instead of a caller workspace.
+ *
+ * Arguments as attn_decode_splitkv, without the workspace.  The scratch holds
+ * FATTN_DECODE_NOALLOC_SCRATCH_BYTES per device; a call that needs more
+ * (B*H*S*(d+1)*4 bytes for S splits, see attn_decode_workspace_bytes) returns
+ * FATTN_ERR_WORKSPACE and enqueues nothing.
+ *
+ * - The scratch is a static device array: every GPU on which the library is
+ *   used holds it until the process exits.  This function allocates nothing
+ *   and calls no allocating routine.
+ * - The first call on a device (with that device current) looks up the
+ *   array's device address once and keeps it; make that first call before
+ *   any stream capture begins.
+ * - All calls share the one array, and each leaves its partials there.  No
+ *   part of it needs to start at zero: a call writes every slot it reads.
+ *   Calls whose executions overlap on the GPU (different streams, or several
+ *   host threads) race on the scratch and give wrong results; order them.
+ */
+#define FATTN_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
+int attn_decode_splitkv_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                void* o, float* lse, const int* seqlens_k,
+                                int B, int H, int Lk, int d, float scale, int num_splits,
+                                void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -50,6 +50,12 @@ std::mutex g_mutex;
 DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+// Library-owned decode scratch for attn_decode_splitkv_noalloc.  Host code
+// must not pass the array's name to a kernel (on the host it names a
+// stand-in, not device memory): its device address is looked up per device.
+__device__ __align__(256) float g_decode_noalloc_scratch[FATTN_DECODE_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+void* g_noalloc_scratch_addr[kMaxDevices] = {};
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Current device, checked to be sm_100 with the kernels' launch attributes set.
@@ -318,6 +324,38 @@ int fattn_device_status(void* stream) {
         return FATTN_ERR_CUDA;
     }
     return v;
+}
+
+int attn_decode_splitkv_noalloc(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                                const int* seqlens_k, int B, int H, int Lk, int d, float scale, int num_splits,
+                                void* stream) {
+    // host-only checks first: nothing is enqueued for a call the scratch cannot hold
+    if (B < 1 || H < 1 || Lk < 1 || num_splits < 0 || (d != 64 && d != 128)) {
+        return attn_decode_splitkv(q, k_cache, v_cache, o, lse, seqlens_k, B, H, Lk, d, scale, num_splits,
+                                   nullptr, 0, stream);
+    }
+    const size_t need = attn_decode_workspace_bytes(B, H, Lk, d, num_splits);
+    if (need == 0 || need > FATTN_DECODE_NOALLOC_SCRATCH_BYTES) return FATTN_ERR_WORKSPACE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return FATTN_ERR_NO_DEVICE;
+    }
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (g_noalloc_scratch_addr[dev] == nullptr) {
+            void* addr = nullptr;
+            if (cudaGetSymbolAddress(&addr, g_decode_noalloc_scratch) != cudaSuccess || addr == nullptr) {
+                cudaGetLastError();
+                return FATTN_ERR_CUDA;
+            }
+            g_noalloc_scratch_addr[dev] = addr;
+        }
+        scratch = g_noalloc_scratch_addr[dev];
+    }
+    return attn_decode_splitkv(q, k_cache, v_cache, o, lse, seqlens_k, B, H, Lk, d, scale, num_splits, scratch,
+                               FATTN_DECODE_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"

@@ -29,6 +29,8 @@ lib.attn_fwd_f32.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i
 lib.attn_fwd_f32.restype = _i
 lib.attn_decode_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz, _vp]
 lib.attn_decode_splitkv.restype = _i
+lib.attn_decode_splitkv_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp]
+lib.attn_decode_splitkv_noalloc.restype = _i
 lib.attn_decode_auto_splits.argtypes = [_i, _i, _i, _i]
 lib.attn_decode_auto_splits.restype = _i
 lib.attn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
@@ -161,6 +163,29 @@ def attn_decode_splitkv(q, k_cache, v_cache, o=None, lse=None, seqlens_k=None, s
                                    _ptr(seqlens_k), B, H, Lk, d, scale, S, _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream()),
            "attn_decode_splitkv")
+    return o, lse
+
+
+def attn_decode_splitkv_noalloc(q, k_cache, v_cache, o=None, lse=None, seqlens_k=None, scale=None,
+                                num_splits=0):
+    """Split-KV decode whose split partials live in the library's own static
+    scratch (for callers that cannot allocate device memory); o and lse are
+    still the caller's.  Same results as attn_decode_splitkv."""
+    _want(q, torch.bfloat16, 4, "q")
+    _want(k_cache, torch.bfloat16, 4, "k_cache")
+    _want(v_cache, torch.bfloat16, 4, "v_cache")
+    B, H, _, d = q.shape
+    Lk = k_cache.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if seqlens_k is not None:
+        _want(seqlens_k, torch.int32, 1, "seqlens_k")
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    _check(lib.attn_decode_splitkv_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
+                                           _ptr(seqlens_k), B, H, Lk, d, scale, int(num_splits), _stream()),
+           "attn_decode_splitkv_noalloc")
     return o, lse
 
 

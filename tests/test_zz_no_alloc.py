@@ -1,0 +1,70 @@
+"""The decode entry point for callers that cannot allocate device memory.
+
+attn_decode_splitkv_noalloc keeps its split partials in a scratch array that
+is part of the library, so a caller that only owns its inputs and outputs (a
+plugin handed buffers by its host application, a service under a fixed memory
+budget) can run split-KV decode without a workspace.  These checks call it
+through the C ABI and compare it with attn_decode_splitkv, which takes a
+caller workspace, on two calls in a row with different shapes (the second call
+must not depend on what the first left in the shared scratch).  The file sorts
+last so that a run stopping at the first failure has run every other test.
+"""
+import numpy as np
+import pytest
+import torch
+
+from io_aware_exact_34_b200 import synth
+from tests._compare import BF16_O_MAXABS, LSE_ABS
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fl():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from io_aware_exact_34_b200 import build
+    build.build()
+    from io_aware_exact_34_b200 import fattn
+    return fattn
+
+
+def _inputs(B, H, Lk, d, seed):
+    q, _, _ = synth.random_qkv(B, H, 1, 1, d, "bf16", seed=seed)
+    _, k, v = synth.random_qkv(B, H, 1, Lk, d, "bf16", seed=seed + 1)
+    g = torch.Generator().manual_seed(seed)
+    seqlens = torch.randint(0, Lk + 1, (B,), generator=g, dtype=torch.int32)
+    seqlens[0] = Lk
+    seqlens[-1] = 0
+    return q.cuda(), k.cuda(), v.cuda(), seqlens.cuda()
+
+
+def test_noalloc_decode_matches_workspace_decode(fl):
+    for B, H, Lk, d, S, seed in [(6, 8, 5000, 128, 16, 21), (3, 4, 700, 64, 5, 22)]:
+        q, k, v, seqlens = _inputs(B, H, Lk, d, seed)
+        o_ref, lse_ref = fl.attn_decode_splitkv(q, k, v, seqlens_k=seqlens, num_splits=S)
+        o, lse = fl.attn_decode_splitkv_noalloc(q, k, v, seqlens_k=seqlens, num_splits=S)
+        torch.cuda.synchronize()
+        o_ref, o = o_ref.float().cpu().numpy(), o.float().cpu().numpy()
+        lse_ref, lse = lse_ref.cpu().numpy(), lse.cpu().numpy()
+        assert np.abs(o - o_ref).max() <= BF16_O_MAXABS
+        empty = np.isneginf(lse_ref)
+        assert np.array_equal(np.isneginf(lse), empty)
+        assert np.abs(lse[~empty] - lse_ref[~empty]).max() <= LSE_ABS
+
+
+def test_noalloc_rejects_more_than_its_scratch(fl):
+    # 16 x 32 heads x 64 splits x 129 floats x 4 B = 16.9 MB > 16 MiB of scratch;
+    # the tensors are full size, so the call would be valid with a workspace
+    B, H, Lk, d, S = 16, 32, 8192, 128, 64
+    need = fl.attn_decode_workspace_bytes(B, H, Lk, d, S)
+    assert need > (16 << 20)
+    q = torch.zeros((B, H, 1, d), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((B, H, Lk, d), dtype=torch.bfloat16, device="cuda")
+    o = torch.empty_like(q)
+    status = fl.lib.attn_decode_splitkv_noalloc(q.data_ptr(), kv.data_ptr(), kv.data_ptr(), o.data_ptr(), None,
+                                                None, B, H, Lk, d, 0.1, S, None)
+    assert status == fl.FATTN_ERR_WORKSPACE
+    o2, _ = fl.attn_decode_splitkv_noalloc(q, kv, kv, num_splits=8)   # fits: 2.1 MB
+    torch.cuda.synchronize()
+    assert torch.all(o2 == 0)
