@@ -19,6 +19,7 @@ data path (weak scaling); the time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -266,25 +267,31 @@ def run_ours(args, world, rank, local):
         fattn.attn_fwd(q, k, v, o=o, lse=lse, scale=w.scale, causal=w.causal,
                        window_left=w.window_left, window_right=w.window_right)
 
-    with ClockSampler(local) as clk:
+    if args.no_headline:
+        ms, clocks, value, roofline = float("nan"), None, None, None
+    elif args.no_clocks:
         ms = timed(world, step, args.steps, args.warmup)
-        # keep the same work running for about a second so the sampler sees it
-        t_end = time.perf_counter() + 1.0
-        while time.perf_counter() < t_end:
-            for _ in range(20):
-                step()
-            torch.cuda.synchronize()
-    clocks = clk.summary()
-
-    value = world * flops / (ms * 1e-3) / 1e12
-    achieved = flops / (ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": recorded_traffic(PREFILL_KERNEL, w.name),
-                "peak_source": f"{peak_src} bf16 dense (burst)", "kernel": PREFILL_KERNEL}
+        clocks = None
+    else:
+        with ClockSampler(local) as clk:
+            ms = timed(world, step, args.steps, args.warmup)
+            # keep the same work running for about a second so the sampler sees it
+            t_end = time.perf_counter() + 1.0
+            while time.perf_counter() < t_end:
+                for _ in range(20):
+                    step()
+                torch.cuda.synchronize()
+        clocks = clk.summary()
+    if not args.no_headline:
+        value = world * flops / (ms * 1e-3) / 1e12
+        achieved = flops / (ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": achieved / peaks["bf16_tflops"], "traffic": recorded_traffic(PREFILL_KERNEL, w.name),
+                    "peak_source": f"{peak_src} bf16 dense (burst)", "kernel": PREFILL_KERNEL}
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.no_headline:
         qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
         oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
@@ -310,6 +317,8 @@ def run_ours(args, world, rank, local):
     decode = None
     if not args.no_decode:
         wd = synth.WORKLOADS[DECODE]
+        if args.decode_batch > 0:
+            wd = dataclasses.replace(wd, B=args.decode_batch, name=f"{wd.name}_b{args.decode_batch}")
         dq, dk, dv = synth.make_inputs(wd, device=dev, seed=wd.seed + rank)
         do = torch.empty_like(dq)
         dl = torch.empty((wd.B, wd.H), dtype=torch.float32, device=dev)
@@ -384,6 +393,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-headline", action="store_true", help="skip the headline prefill (profiling runs)")
     ap.add_argument("--decode-batch", type=int, default=0, help="override the decode batch (profiling runs)")
+    ap.add_argument("--no-clocks", action="store_true", help="no nvidia-smi sampling or soak (profiling runs)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
