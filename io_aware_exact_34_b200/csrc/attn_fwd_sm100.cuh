@@ -85,8 +85,7 @@ struct FwdParams {
 // The two Q tiles of one work item and the KV tiles they visit.
 struct PairTiles {
     int bh;
-    long long q_first[2], q_last[2];
-    bool exists[2];
+    int q_first[2];
     int lo_t[2], hi_t[2];
     int lo, hi;  // union range
 };
@@ -106,12 +105,11 @@ __device__ __forceinline__ PairTiles pair_tiles(const FwdParams& p, const Band& 
     ts.hi = 0;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-        const long long q_first = static_cast<long long>(2 * pair + t) * 128;
+        const int q_first = (2 * pair + t) * 128;
+        const int q_last = q_first + 127 < p.Lq - 1 ? q_first + 127 : p.Lq - 1;
         ts.q_first[t] = q_first;
-        ts.exists[t] = q_first < p.Lq;
-        ts.q_last[t] = q_first + 127 < p.Lq - 1 ? q_first + 127 : p.Lq - 1;
         int lo = 0, hi = 0;
-        if (ts.exists[t]) kv_tile_range(band, q_first, ts.q_last[t], 128, &lo, &hi);
+        if (q_first < p.Lq) kv_tile_range(band, q_first, q_last, 128, &lo, &hi);
         ts.lo_t[t] = lo;
         ts.hi_t[t] = hi;
         if (lo < hi) {
@@ -162,6 +160,61 @@ __device__ __forceinline__ RowPlan row_plan(const FwdParams& p, int item, int t,
     rp.full_lo = clamp_int(flo);
     rp.full_hi = clamp_int(fhi);
     return rp;
+}
+
+// Exponentials of one 128-score row: p_c = 2^(s_c * c_log2 - m_safe), packed
+// to bf16 pairs in pk (key 2i in the low half of pk[i / 32][i % 32]); returns
+// the fp32 row sum of the p_c.  Scores are scaled and shifted in packed f32x2
+// FMAs.  On tiles with no masked position (kUnmasked) one pair in every
+// kPolyExp2Every goes through exp2_poly_pair on the FMA pipe, the rest through
+// the MUFU ex2; masked tiles use ex2 only, so masked scores (-inf) give
+// exactly 0.  Measured on B200 at d = 128 the MUFU is not the limit (any
+// polynomial share was slower), so the default share is zero.
+#ifndef FATTN_POLY_EXP2_EVERY
+#define FATTN_POLY_EXP2_EVERY 0
+#endif
+constexpr int kPolyExp2Every = FATTN_POLY_EXP2_EVERY;
+constexpr int kPolyExp2Mod = kPolyExp2Every > 0 ? kPolyExp2Every : 1;
+
+template <bool kUnmasked>
+__device__ __forceinline__ float softmax_tile_probs(const uint32_t (&sr)[4][32], uint32_t (&pk)[2][32], float c_log2,
+                                                    float m_safe) {
+    const uint64_t scale2 = f2_pack(c_log2, c_log2);
+    const uint64_t shift2 = f2_pack(-m_safe, -m_safe);
+    uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};  // independent partial sums: no long add chain
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const int c = 2 * i;
+        const uint64_t s2 = f2_pack(__uint_as_float(sr[c >> 5][c & 31]), __uint_as_float(sr[c >> 5][(c & 31) + 1]));
+        const uint64_t x2 = f2_fma(s2, scale2, shift2);
+        uint64_t p2;
+        if (kUnmasked && kPolyExp2Every > 0 && (i % kPolyExp2Mod) == kPolyExp2Mod - 1) {
+            p2 = exp2_poly_pair(x2);
+        } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
+        }
+        sum2[i & 3] = f2_add(sum2[i & 3], p2);
+        float p0, p1;
+        f2_unpack(p2, p0, p1);
+        pk[i >> 5][i & 31] = pack_bf16x2(p0, p1);
+    }
+    const uint64_t s01 = f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3]));
+    float lo, hi;
+    f2_unpack(s01, lo, hi);
+    return lo + hi;
+}
+
+// Row max of 128 scores with four independent 3-input max chains.
+__device__ __forceinline__ float row_max128(const uint32_t (&sr)[4][32]) {
+    float m[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const int c = 2 * i;
+        m[i & 3] = fmax3(m[i & 3], __uint_as_float(sr[c >> 5][c & 31]), __uint_as_float(sr[c >> 5][(c & 31) + 1]));
+    }
+    return fmax3(m[0], m[1], fmaxf(m[2], m[3]));
 }
 
 template <int D>
@@ -242,7 +295,7 @@ __global__ void __launch_bounds__(384, 1)
                 for (int t = 0; t < 2; ++t)
                     for (int c = 0; c < T::NCHUNK; ++c)
                         tma_load_3d(sQ + t * T::TILE_BYTES + c * T::CHUNK_BYTES, &tm_q, q_full, c * 64,
-                                    static_cast<int>(ts.q_first[t]), ts.bh);
+                                    ts.q_first[t], ts.bh);
                 ++q_round;
                 for (int j = ts.lo; j < ts.hi && ok; ++j) {
                     for (int kv = 0; kv < 2; ++kv) {
@@ -302,25 +355,27 @@ __global__ void __launch_bounds__(384, 1)
                             ++p_cnt[t];
                             if (!ok) break;
                             tc_fence_after_sync();
-                            const uint32_t vbase = sRing + (rV % T::NSTAGE) * T::TILE_BYTES;
+                            const uint32_t v_lo = sdesc_lo(sRing + (rV % T::NSTAGE) * T::TILE_BYTES, T::CHUNK_BYTES);
                             const uint32_t first = (j - 1 == ts.lo_t[t]) ? 1u : 0u;
 #pragma unroll
                             for (int ks = 0; ks < 8; ++ks) {
-                                const uint64_t bdesc = sdesc_sw128(vbase + ks * 2048, T::CHUNK_BYTES, 1024);
-                                mma_bf16_ts(tmem + T::tm_o(t), tmem + T::tm_s(t) + ks * 8, bdesc, idesc_pv,
+                                // 16 keys = 16 rows of 128 B further into the V tile
+                                mma_bf16_ts(tmem + T::tm_o(t), tmem + T::tm_s(t) + ks * 8,
+                                            sdesc_from_lo(v_lo + ks * (2048 >> 4)), idesc_pv,
                                             (first && ks == 0) ? 0u : 1u);
                             }
                             if (j - 1 == ts.hi_t[t] - 1) mma_commit(o_full0 + 8 * t);
                         }
                         // S_t = Q_t K_j^T
                         if (haveK && j >= ts.lo_t[t] && j < ts.hi_t[t]) {
-                            const uint32_t kbase = sRing + (rK % T::NSTAGE) * T::TILE_BYTES;
-                            const uint32_t qbase = sQ + t * T::TILE_BYTES;
+                            const uint32_t k_lo = sdesc_lo(sRing + (rK % T::NSTAGE) * T::TILE_BYTES, 16);
+                            const uint32_t q_lo = sdesc_lo(sQ + t * T::TILE_BYTES, 16);
 #pragma unroll
                             for (int ks = 0; ks < D / 16; ++ks) {
-                                const uint32_t off = (ks / 4) * T::CHUNK_BYTES + (ks % 4) * 32;
-                                mma_bf16_ss(tmem + T::tm_s(t), sdesc_sw128(qbase + off, 16, 1024),
-                                            sdesc_sw128(kbase + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+                                // 16 elements = 32 B along the swizzled row; 64 elements = next 16 KB column
+                                const uint32_t off = ((ks / 4) * T::CHUNK_BYTES + (ks % 4) * 32) >> 4;
+                                mma_bf16_ss(tmem + T::tm_s(t), sdesc_from_lo(q_lo + off), sdesc_from_lo(k_lo + off),
+                                            idesc_s, ks > 0 ? 1u : 0u);
                             }
                             mma_commit(s_full0 + 8 * t);
                         }
@@ -378,17 +433,15 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) reg_fence(sr[q4]);
                 const int k0 = j * 128;
-                if (!(k0 >= rp.full_lo && k0 + 127 <= rp.full_hi)) {
+                const bool full_tile = k0 >= rp.full_lo && k0 + 127 <= rp.full_hi;
+                if (!full_tile) {
                     // §5.2: the boundary mask goes on before the softmax
                     const int lo_col = rp.key_lo - k0, hi_col = rp.key_hi - k0;
 #pragma unroll
                     for (int c = 0; c < 128; ++c)
                         if (c < lo_col || c > hi_col) sr[c >> 5][c & 31] = __float_as_uint(-CUDART_INF_F);
                 }
-                float mx = -CUDART_INF_F;
-#pragma unroll
-                for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c >> 5][c & 31]));
-                const float mx_s = mx * c_log2;
+                const float mx_s = row_max128(sr) * c_log2;
                 float alpha = 1.f;
                 bool resc = false;
                 if (mx_s > m_used + kRescaleSlack) {
@@ -398,15 +451,12 @@ __global__ void __launch_bounds__(384, 1)
                     l *= alpha;
                 }
                 const float m_safe = (m_used == -CUDART_INF_F) ? 0.f : m_used;
-                float rowsum = 0.f;
                 uint32_t pk[2][32];
-#pragma unroll
-                for (int c = 0; c < 128; c += 2) {
-                    const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c >> 5][c & 31]), c_log2, -m_safe));
-                    const float p1 = fast_exp2(fmaf(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]), c_log2, -m_safe));
-                    rowsum += p0 + p1;
-                    pk[c >> 6][(c & 63) >> 1] = pack_bf16x2(p0, p1);
-                }
+                float rowsum;
+                if (full_tile)
+                    rowsum = softmax_tile_probs<true>(sr, pk, c_log2, m_safe);
+                else
+                    rowsum = softmax_tile_probs<false>(sr, pk, c_log2, m_safe);
                 l += rowsum;
                 tmem_st32(taddr_s, pk[0]);
                 tmem_st32(taddr_s + 32, pk[1]);
