@@ -48,10 +48,17 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_digest() -> str:
+KERNEL_SOURCES = {
+    "attn_fwd_sm100_kernel": ["attn_fwd_sm100.cuh", "sched.cuh", "dev_prims.cuh"],
+    "decode_split_kernel": ["decode_splitkv.cuh", "dev_prims.cuh"],
+}
+
+
+def kernel_source_digest(kernel: str) -> str:
+    """Digest of the source files a kernel is compiled from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "io_aware_exact_34_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -66,7 +73,7 @@ def recorded_traffic(kernel: str, workload: str):
     with open(path) as f:
         rec = json.load(f)
     ent = rec.get(kernel, {}).get(workload)
-    if not ent or ent.get("source_digest") != kernel_source_digest():
+    if not ent or ent.get("source_digest") != kernel_source_digest(kernel):
         return None
     return ent.get("bytes_per_launch")
 
@@ -149,13 +156,21 @@ def barrier(world):
 
 
 def max_over_ranks(world, value: float) -> float:
+    """The slowest rank's time: every rank gets the max (an all-reduce on the
+    process group's device, CPU tensors for gloo)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_seed(base_seed: int, rank: int) -> int:
+    """Each replica draws its own inputs of the same shape (weak scaling)."""
+    return base_seed + rank
 
 
 def timed(world, fn, steps, warmup):
@@ -259,7 +274,7 @@ def run_ours(args, world, rank, local):
     # ---------------------------------------------------------------- headline prefill
     w = synth.WORKLOADS[HEADLINE]
     flops, counts = prefill_flops(fattn, w)
-    q, k, v = synth.make_inputs(w, device=dev, seed=w.seed + rank)
+    q, k, v = synth.make_inputs(w, device=dev, seed=replica_seed(w.seed, rank))
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev)
 
@@ -319,7 +334,7 @@ def run_ours(args, world, rank, local):
         wd = synth.WORKLOADS[DECODE]
         if args.decode_batch > 0:
             wd = dataclasses.replace(wd, B=args.decode_batch, name=f"{wd.name}_b{args.decode_batch}")
-        dq, dk, dv = synth.make_inputs(wd, device=dev, seed=wd.seed + rank)
+        dq, dk, dv = synth.make_inputs(wd, device=dev, seed=replica_seed(wd.seed, rank))
         do = torch.empty_like(dq)
         dl = torch.empty((wd.B, wd.H), dtype=torch.float32, device=dev)
         ws = torch.empty(fattn.attn_decode_workspace_bytes(wd.B, wd.H, wd.Lk, wd.d, wd.num_splits),
@@ -349,7 +364,7 @@ def run_ours(args, world, rank, local):
         for name in EXTRA:
             we = synth.WORKLOADS[name]
             f_e, c_e = prefill_flops(fattn, we)
-            eq, ek, ev = synth.make_inputs(we, device=dev, seed=we.seed + rank)
+            eq, ek, ev = synth.make_inputs(we, device=dev, seed=replica_seed(we.seed, rank))
             eo = torch.empty_like(eq)
             el = torch.empty((we.B, we.H, we.Lq), dtype=torch.float32, device=dev)
 

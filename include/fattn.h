@@ -160,6 +160,17 @@ const char* fattn_status_string(int status);
 int fattn_device_status(void* stream);
 
 /*
+ * fattn_debug_inject_stall -- test hook for the failure path.  With on != 0
+ * the next attn_fwd / attn_fwd_counted launch (only that one) leaves the
+ * first K tile of CTA 0 undelivered: nothing is loaded and nothing faults,
+ * the waits that depend on it run out their time limit (about 2 s), and the
+ * kernel records FATTN_ERR_TIMEOUT in the device status word, drains its
+ * in-flight copies and MMAs, frees its tensor memory and exits.  That launch's
+ * O and LSE are garbage; later launches are unaffected.
+ */
+int fattn_debug_inject_stall(int on);
+
+/*
  * attn_decode_splitkv_noalloc -- attn_decode_splitkv for callers that cannot
  * allocate device memory.  The pages have no counterpart to this entry point;
  * it exists for the library's users, not for the method.

@@ -80,6 +80,7 @@ struct FwdParams {
     float scale_log2;  // scale * log2(e)
     int causal, window_left, window_right;
     int n_pairs, n_items;
+    int inject_stall;  // test hook: CTA 0 never delivers its first K tile
 };
 
 // The two Q tiles of one work item and the KV tiles they visit.
@@ -303,6 +304,12 @@ __global__ void __launch_bounds__(384, 1)
                         if (use > 0) {
                             ok = mbar_wait(kv_empty0 + 8 * slot, (use - 1) & 1u, abort_flag, status, -6);
                             if (!ok) break;
+                        }
+                        if (p.inject_stall && blockIdx.x == 0 && ring == 0) {
+                            // Test hook: this tile is never loaded, so every wait
+                            // that depends on it runs out its time limit.
+                            ++ring;
+                            continue;
                         }
                         const uint32_t fb = kv_full0 + 8 * slot;
                         mbar_arrive_expect_tx(fb, T::TILE_BYTES);

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -49,6 +50,7 @@ bool fwd_register_pool_ok() {
 std::mutex g_mutex;
 DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::atomic<int> g_inject_stall{0};
 
 // Library-owned decode scratch for attn_decode_splitkv_noalloc.  Host code
 // must not pass the array's name to a kernel (on the host it names a
@@ -164,6 +166,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.window_right = wr < 0 ? -1 : wr;
     p.n_pairs = static_cast<int>(n_pairs);
     p.n_items = static_cast<int>(n_items);
+    p.inject_stall = g_inject_stall.exchange(0);
     const int grid = static_cast<int>(n_items < di.num_sms ? n_items : di.num_sms);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (d == 128)
@@ -310,6 +313,11 @@ const char* fattn_status_string(int status) {
         case FATTN_ERR_NO_DEVICE: return "FATTN_ERR_NO_DEVICE: no usable sm_100 device";
         default: return "unknown fattn status";
     }
+}
+
+int fattn_debug_inject_stall(int on) {
+    g_inject_stall.store(on ? 1 : 0);
+    return FATTN_OK;
 }
 
 int fattn_device_status(void* stream) {

@@ -41,6 +41,8 @@ lib.fattn_status_string.argtypes = [_i]
 lib.fattn_status_string.restype = ctypes.c_char_p
 lib.fattn_device_status.argtypes = [_vp]
 lib.fattn_device_status.restype = _i
+lib.fattn_debug_inject_stall.argtypes = [_i]
+lib.fattn_debug_inject_stall.restype = _i
 
 FATTN_OK = 0
 FATTN_ERR_INVALID_ARG = -1
@@ -199,6 +201,11 @@ def attn_count_blocks(Lq, Lk, causal=False, window_left=-1, window_right=-1, blo
 
 def fattn_device_status() -> int:
     return lib.fattn_device_status(_stream())
+
+
+def fattn_debug_inject_stall(on: bool = True) -> None:
+    """Test hook: the next prefill launch lets its bounded waits run out."""
+    _check(lib.fattn_debug_inject_stall(int(bool(on))), "fattn_debug_inject_stall")
 
 
 def status_string(status: int) -> str:
