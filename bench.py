@@ -36,6 +36,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 HEADLINE = "causal_4k"
 DECODE = "decode_32k"
 EXTRA = ["window_bidir_32k", "window_causal_32k", "causal_64k_qscale"]
+VARLEN_SEQS, VARLEN_MIN, VARLEN_MAX, VARLEN_H = 32, 256, 4096, 16  # packed batch of causal requests
 PREFILL_KERNEL = "attn_fwd_sm100_kernel"
 
 
@@ -381,6 +382,28 @@ def run_ours(args, world, rank, local):
                            "config": we.describe()}
             del eq, ek, ev, eo, el
             torch.cuda.empty_cache()
+
+    # ---------------------------------------------------------------- packed variable-length prefill
+    if not args.no_extra:
+        lens = synth.varlen_lengths(VARLEN_SEQS, VARLEN_MIN, VARLEN_MAX, seed=replica_seed(6, rank))
+        vq, vk, vv, cuq, cuk = synth.make_varlen_inputs(lens, lens, VARLEN_H, 128, seed=replica_seed(6, rank), device=dev)
+        vo = torch.empty_like(vq)
+        vl = torch.empty((VARLEN_H, vq.shape[0]), dtype=torch.float32, device=dev)
+        f_v = sum(4.0 * 128 * fattn.attn_count_blocks(L, L, True, -1, -1, 128, 128)["pairs"] * VARLEN_H for L in lens)
+
+        def vstep():
+            fattn.attn_fwd_varlen(vq, vk, vv, cuq, cuk, max(lens), o=vo, lse=vl, causal=True)
+
+        vsteps = max(3, min(args.steps, 10))
+        vms = timed(world, vstep, vsteps, 2)
+        tf = f_v / (vms * 1e-3) / 1e12
+        extra["varlen_causal_32seq"] = {"value": world * tf, "unit": "TFLOP/s", "ms_per_step": vms, "steps": vsteps,
+                                        "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
+                                        "config": {"workload": "varlen_causal_32seq", "num_seqs": VARLEN_SEQS,
+                                                   "seqlen_range": [VARLEN_MIN, VARLEN_MAX], "total_tokens": int(sum(lens)),
+                                                   "H": VARLEN_H, "d": 128, "causal": True, "layout": "packed [total, H, d]"}}
+        del vq, vk, vv, vo, vl
+        torch.cuda.empty_cache()
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:

@@ -93,6 +93,38 @@ int attn_fwd_counted(const void* q, const void* k, const void* v, void* o, float
                      unsigned long long* kv_tiles_visited, void* stream);
 
 /*
+ * attn_fwd_varlen -- attn_fwd over a packed batch of sequences of different
+ * lengths (the sliding-window FlashAttention prefill page §8.1: requests of
+ * different lengths share one launch, each sequence with its own clipped KV
+ * range, instead of padding every request to a common length).
+ *
+ *   q, o          device, bf16 [total_q, H, d]: the tokens of all sequences
+ *                 back to back, token-major; 16-byte aligned
+ *   k, v          device, bf16 [total_k, H, d]
+ *   lse           device, fp32 [H, total_q], or NULL
+ *   cu_seqlens_q  device, int32 [num_seqs + 1], non-decreasing: sequence b
+ *                 owns query tokens [cu_seqlens_q[b], cu_seqlens_q[b+1])
+ *   cu_seqlens_k  device, int32 [num_seqs + 1]: likewise for the keys/values
+ *   max_seqlen_q  at least every sequence's query length (query rows beyond
+ *                 it are not computed)
+ * The mask applies per sequence exactly as in attn_fwd, with Lq and Lk the
+ * sequence's own lengths (bottom-right alignment when they differ).  Offsets
+ * read from cu_seqlens are clamped into [0, total], so no access leaves the
+ * tensors; a sequence with no query token writes nothing.
+ */
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs, int H,
+                    int total_q, int total_k, int max_seqlen_q, int d, float scale,
+                    int causal, int window_left, int window_right, void* stream);
+
+/* attn_fwd_varlen that also counts the KV tiles visited (see attn_fwd_counted). */
+int attn_fwd_varlen_counted(const void* q, const void* k, const void* v, void* o, float* lse,
+                            const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs, int H,
+                            int total_q, int total_k, int max_seqlen_q, int d, float scale,
+                            int causal, int window_left, int window_right,
+                            unsigned long long* kv_tiles_visited, void* stream);
+
+/*
  * attn_fwd_f32 -- the same operation on fp32 Q/K/V/O with fp32 arithmetic on
  * the CUDA cores (no tensor-core rounding), for exactness checks.  Arguments
  * as attn_fwd with fp32 tensors; d in {64, 128}; lse nullable.

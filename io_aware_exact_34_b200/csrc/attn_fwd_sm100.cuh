@@ -81,11 +81,47 @@ struct FwdParams {
     int causal, window_left, window_right;
     int n_pairs, n_items;
     int inject_stall;  // test hook: CTA 0 never delivers its first K tile
+    // packed variable-length batches (B = number of sequences): sequence b
+    // owns tokens [cu_q[b], cu_q[b+1]) of Q/O and [cu_k[b], cu_k[b+1]) of K/V
+    const int* cu_q;
+    const int* cu_k;
+    int total_q, total_k;
 };
+
+// The sequence and head of one work item: its pair index, token offsets and
+// lengths.  Dense batches: offsets 0, lengths Lq / Lk, tensors indexed by bh.
+struct ItemSeq {
+    int pair, bh, h;
+    int q_start, k_start;  // first token of the sequence (packed batches)
+    int len_q, len_k;
+};
+
+template <bool kVarlen>
+__device__ __forceinline__ ItemSeq item_seq(const FwdParams& p, int item) {
+    ItemSeq sq;
+    const int BH = p.B * p.H;
+    sq.pair = p.n_pairs - 1 - item / BH;
+    sq.bh = item % BH;
+    sq.h = sq.bh % p.H;
+    if constexpr (kVarlen) {
+        // clamp the caller's offsets into the packed tensors: every access stays in bounds
+        const int b = sq.bh / p.H;
+        auto clampi = [](int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); };
+        sq.q_start = clampi(__ldg(p.cu_q + b), 0, p.total_q);
+        sq.len_q = clampi(__ldg(p.cu_q + b + 1), sq.q_start, p.total_q) - sq.q_start;
+        sq.k_start = clampi(__ldg(p.cu_k + b), 0, p.total_k);
+        sq.len_k = clampi(__ldg(p.cu_k + b + 1), sq.k_start, p.total_k) - sq.k_start;
+    } else {
+        sq.q_start = sq.k_start = 0;
+        sq.len_q = p.Lq;
+        sq.len_k = p.Lk;
+    }
+    return sq;
+}
 
 // The two Q tiles of one work item and the KV tiles they visit.
 struct PairTiles {
-    int bh;
+    int bh, h, q_start, k_start;
     int q_first[2];
     int lo_t[2], hi_t[2];
     int lo, hi;  // union range
@@ -97,20 +133,24 @@ __device__ __forceinline__ int snake_item(int round, int cta, int grid) {
     return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
 }
 
-__device__ __forceinline__ PairTiles pair_tiles(const FwdParams& p, const Band& band, int item) {
+template <bool kVarlen>
+__device__ __forceinline__ PairTiles pair_tiles(const FwdParams& p, int item) {
     PairTiles ts;
-    const int BH = p.B * p.H;
-    const int pair = p.n_pairs - 1 - item / BH;
-    ts.bh = item % BH;
+    const ItemSeq sq = item_seq<kVarlen>(p, item);
+    const Band band = make_band(sq.len_q, sq.len_k, p.causal, p.window_left, p.window_right);
+    ts.bh = sq.bh;
+    ts.h = sq.h;
+    ts.q_start = sq.q_start;
+    ts.k_start = sq.k_start;
     ts.lo = 0x7fffffff;
     ts.hi = 0;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-        const int q_first = (2 * pair + t) * 128;
-        const int q_last = q_first + 127 < p.Lq - 1 ? q_first + 127 : p.Lq - 1;
+        const int q_first = (2 * sq.pair + t) * 128;
+        const int q_last = q_first + 127 < sq.len_q - 1 ? q_first + 127 : sq.len_q - 1;
         ts.q_first[t] = q_first;
         int lo = 0, hi = 0;
-        if (q_first < p.Lq) kv_tile_range(band, q_first, q_last, 128, &lo, &hi);
+        if (q_first < sq.len_q) kv_tile_range(band, q_first, q_last, 128, &lo, &hi);
         ts.lo_t[t] = lo;
         ts.hi_t[t] = hi;
         if (lo < hi) {
@@ -126,7 +166,8 @@ __device__ __forceinline__ PairTiles pair_tiles(const FwdParams& p, const Band& 
 // tile range of its Q tile, the key bounds of its row and the key window in
 // which a tile needs no mask at all (absolute key indices, clamped to int).
 struct RowPlan {
-    long long orow;   // row index into O / LSE ([B*H*Lq])
+    long long o_off;    // element offset of this row in O
+    long long lse_off;  // element offset of this row in LSE
     int lo, hi;       // KV tile range of the Q tile
     int key_lo, key_hi;   // allowed keys of this row: [key_lo, key_hi]
     int full_lo, full_hi; // a tile [k0, k0+127] is unmasked iff k0 >= full_lo && k0+127 <= full_hi
@@ -137,18 +178,25 @@ __device__ __forceinline__ int clamp_int(long long x) {
     return static_cast<int>(x < -(1LL << 30) ? -(1LL << 30) : (x > (1LL << 30) ? (1LL << 30) : x));
 }
 
+template <int D, bool kVarlen>
 __device__ __forceinline__ RowPlan row_plan(const FwdParams& p, int item, int t, int row) {
     RowPlan rp;
-    const Band band = make_band(p.Lq, p.Lk, p.causal, p.window_left, p.window_right);
-    const int BH = p.B * p.H;
-    const int pair = p.n_pairs - 1 - item / BH;
-    const int bh = item % BH;
-    const long long q_first = static_cast<long long>(2 * pair + t) * 128;
-    const long long q_last = q_first + 127 < p.Lq - 1 ? q_first + 127 : p.Lq - 1;
+    const ItemSeq sq = item_seq<kVarlen>(p, item);
+    const Band band = make_band(sq.len_q, sq.len_k, p.causal, p.window_left, p.window_right);
+    const long long q_first = static_cast<long long>(2 * sq.pair + t) * 128;
+    const long long q_last = q_first + 127 < sq.len_q - 1 ? q_first + 127 : sq.len_q - 1;
     const long long i = q_first + row;
-    rp.tile_exists = q_first < p.Lq;
-    rp.valid = i < p.Lq;
-    rp.orow = static_cast<long long>(bh) * p.Lq + i;
+    rp.tile_exists = q_first < sq.len_q;
+    rp.valid = i < sq.len_q;
+    if constexpr (kVarlen) {
+        // packed layout: O [total_q, H, D], LSE [H, total_q]
+        const long long tok = sq.q_start + i;
+        rp.o_off = (tok * p.H + sq.h) * D;
+        rp.lse_off = static_cast<long long>(sq.h) * p.total_q + tok;
+    } else {
+        rp.o_off = (static_cast<long long>(sq.bh) * p.Lq + i) * D;
+        rp.lse_off = static_cast<long long>(sq.bh) * p.Lq + i;
+    }
     rp.lo = rp.hi = 0;
     if (rp.tile_exists) kv_tile_range(band, q_first, q_last, 128, &rp.lo, &rp.hi);
     int lo_col, hi_col;
@@ -218,7 +266,7 @@ __device__ __forceinline__ float row_max128(const uint32_t (&sr)[4][32]) {
     return fmax3(m[0], m[1], fmaxf(m[2], m[3]));
 }
 
-template <int D>
+template <int D, bool kVarlen>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -277,7 +325,6 @@ __global__ void __launch_bounds__(384, 1)
 
     if (warp < 4) {
       warpgroup_reg_lower<T::REGS_LOW>();
-      const Band band = make_band(p.Lq, p.Lk, p.causal, p.window_left, p.window_right);
       if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -286,7 +333,7 @@ __global__ void __launch_bounds__(384, 1)
             for (int round = 0; ok; ++round) {
                 const int item = snake_item(round, blockIdx.x, gridDim.x);
                 if (item >= p.n_items) break;
-                const PairTiles ts = pair_tiles(p, band, item);
+                const PairTiles ts = pair_tiles<kVarlen>(p, item);
                 if (ts.lo >= ts.hi) continue;
                 if (q_round > 0) {
                     ok = mbar_wait(q_empty, (q_round - 1) & 1u, abort_flag, status, -6);
@@ -296,7 +343,7 @@ __global__ void __launch_bounds__(384, 1)
                 for (int t = 0; t < 2; ++t)
                     for (int c = 0; c < T::NCHUNK; ++c)
                         tma_load_3d(sQ + t * T::TILE_BYTES + c * T::CHUNK_BYTES, &tm_q, q_full, c * 64,
-                                    ts.q_first[t], ts.bh);
+                                    kVarlen ? ts.h : ts.q_first[t], kVarlen ? ts.q_start + ts.q_first[t] : ts.bh);
                 ++q_round;
                 for (int j = ts.lo; j < ts.hi && ok; ++j) {
                     for (int kv = 0; kv < 2; ++kv) {
@@ -315,7 +362,7 @@ __global__ void __launch_bounds__(384, 1)
                         mbar_arrive_expect_tx(fb, T::TILE_BYTES);
                         for (int c = 0; c < T::NCHUNK; ++c)
                             tma_load_3d(sRing + slot * T::TILE_BYTES + c * T::CHUNK_BYTES, kv ? &tm_v : &tm_k, fb,
-                                        c * 64, j * 128, ts.bh);
+                                        c * 64, kVarlen ? ts.h : j * 128, kVarlen ? ts.k_start + j * 128 : ts.bh);
                         ++ring;
                     }
                 }
@@ -339,7 +386,7 @@ __global__ void __launch_bounds__(384, 1)
             for (int round = 0; ok; ++round) {
                 const int item = snake_item(round, blockIdx.x, gridDim.x);
                 if (item >= p.n_items) break;
-                const PairTiles ts = pair_tiles(p, band, item);
+                const PairTiles ts = pair_tiles<kVarlen>(p, item);
                 if (ts.lo >= ts.hi) continue;
                 ok = mbar_wait(q_full, q_round & 1u, abort_flag, status, -6);
                 if (!ok) break;
@@ -414,15 +461,15 @@ __global__ void __launch_bounds__(384, 1)
         for (int round = 0; ok; ++round) {
             const int item = snake_item(round, blockIdx.x, gridDim.x);
             if (item >= p.n_items) break;
-            const RowPlan rp = row_plan(p, item, t, row);
+            const RowPlan rp = row_plan<D, kVarlen>(p, item, t, row);
             if (!rp.tile_exists) continue;
             if (rp.lo >= rp.hi) {
                 // no allowed key for any row of this tile
                 if (rp.valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + rp.orow * D);
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + rp.o_off);
 #pragma unroll
                     for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
-                    if (p.lse) p.lse[rp.orow] = -CUDART_INF_F;
+                    if (p.lse) p.lse[rp.lse_off] = -CUDART_INF_F;
                 }
                 continue;
             }
@@ -492,7 +539,7 @@ __global__ void __launch_bounds__(384, 1)
             if (!ok) break;
             tc_fence_after_sync();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + rp.orow * D;
+            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + rp.o_off;
 #pragma unroll 1
             for (int ch = 0; ch < D / 32; ++ch) {
                 uint32_t orr[32];
@@ -509,7 +556,7 @@ __global__ void __launch_bounds__(384, 1)
                     for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk16[4 * v], pk16[4 * v + 1], pk16[4 * v + 2], pk16[4 * v + 3]);
                 }
             }
-            if (rp.valid && p.lse) p.lse[rp.orow] = l > 0.f ? (m_used + __log2f(l)) * 0.6931471805599453f : -CUDART_INF_F;
+            if (rp.valid && p.lse) p.lse[rp.lse_off] = l > 0.f ? (m_used + __log2f(l)) * 0.6931471805599453f : -CUDART_INF_F;
             if (p.visited && quarter == 0 && lane == 0)
                 atomicAdd(p.visited, static_cast<unsigned long long>(rp.hi - rp.lo));
         }

@@ -37,14 +37,15 @@ struct DeviceInfo {
 // raising warpgroups would wait forever.  Checked against the compiled kernel.
 template <int D>
 bool fwd_register_pool_ok() {
-    cudaFuncAttributes a;
-    if (cudaFuncGetAttributes(&a, attn_fwd_sm100_kernel<D>) != cudaSuccess) {
+    cudaFuncAttributes a, b;
+    if (cudaFuncGetAttributes(&a, attn_fwd_sm100_kernel<D, false>) != cudaSuccess ||
+        cudaFuncGetAttributes(&b, attn_fwd_sm100_kernel<D, true>) != cudaSuccess) {
         cudaGetLastError();
         return false;
     }
     using T = FwdTraits<D>;
-    return static_cast<long long>(a.numRegs) * T::THREADS >=
-           128LL * T::REGS_LOW + 256LL * T::REGS_HIGH;
+    const long long need = 128LL * T::REGS_LOW + 256LL * T::REGS_HIGH;
+    return static_cast<long long>(a.numRegs) * T::THREADS >= need && static_cast<long long>(b.numRegs) * T::THREADS >= need;
 }
 
 std::mutex g_mutex;
@@ -82,8 +83,10 @@ int device_ready(DeviceInfo* out) {
         di.num_sms = sms;
         if (di.sm100) {
             cudaError_t e = cudaSuccess;
-            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128>::SMEM_BYTES);
-            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64>::SMEM_BYTES);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128>::SMEM_BYTES);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64>::SMEM_BYTES);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128>::SMEM_BYTES);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, F32Traits<128>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, F32Traits<64>::SMEM_BYTES);
             if (e != cudaSuccess) {
@@ -135,6 +138,29 @@ int encode_map(CUtensorMap* map, const void* base, int d, long long L, long long
     return r == CUDA_SUCCESS ? FATTN_OK : FATTN_ERR_CUDA;
 }
 
+// Packed [total, H, d] bf16 tensor viewed as (d, H, total): 64-element x
+// 1-head x 128-token boxes land as the same 128-row, 128-byte-swizzled tile.
+int encode_map_packed(CUtensorMap* map, const void* base, int d, int H, long long total) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(total)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
+    cuuint32_t box[3] = {64, 1, 128};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FATTN_OK : FATTN_ERR_CUDA;
+}
+
+template <bool kVarlen>
+int launch_prefill_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
+                          int d, int grid, cudaStream_t s) {
+    if (d == 128)
+        attn_fwd_sm100_kernel<128, kVarlen><<<grid, FwdTraits<128>::THREADS, FwdTraits<128>::SMEM_BYTES, s>>>(mq, mk, mv, p);
+    else
+        attn_fwd_sm100_kernel<64, kVarlen><<<grid, FwdTraits<64>::THREADS, FwdTraits<64>::SMEM_BYTES, s>>>(mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? FATTN_OK : FATTN_ERR_CUDA;
+}
+
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq, int Lk, int d,
                float scale, int causal, int wl, int wr, unsigned long long* visited, void* stream) {
     int st = check_prefill(q, k, v, o, lse, B, H, Lq, Lk, d, scale);
@@ -167,13 +193,55 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.n_pairs = static_cast<int>(n_pairs);
     p.n_items = static_cast<int>(n_items);
     p.inject_stall = g_inject_stall.exchange(0);
+    p.cu_q = p.cu_k = nullptr;
+    p.total_q = p.total_k = 0;
     const int grid = static_cast<int>(n_items < di.num_sms ? n_items : di.num_sms);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (d == 128)
-        attn_fwd_sm100_kernel<128><<<grid, FwdTraits<128>::THREADS, FwdTraits<128>::SMEM_BYTES, s>>>(mq, mk, mv, p);
-    else
-        attn_fwd_sm100_kernel<64><<<grid, FwdTraits<64>::THREADS, FwdTraits<64>::SMEM_BYTES, s>>>(mq, mk, mv, p);
-    return cudaGetLastError() == cudaSuccess ? FATTN_OK : FATTN_ERR_CUDA;
+    return launch_prefill_kernel<false>(mq, mk, mv, p, d, grid, static_cast<cudaStream_t>(stream));
+}
+
+int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_q, const int* cu_k,
+                      int nseq, int H, int total_q, int total_k, int max_seqlen_q, int d, float scale, int causal,
+                      int wl, int wr, unsigned long long* visited, void* stream) {
+    if (!cu_q || !cu_k) return FATTN_ERR_INVALID_ARG;
+    if (nseq < 1 || max_seqlen_q < 1) return FATTN_ERR_INVALID_ARG;
+    int st = check_prefill(q, k, v, o, lse, nseq, H, total_q, total_k, d, scale);
+    if (st != FATTN_OK) return st;
+    if ((reinterpret_cast<uintptr_t>(cu_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_k) & 3u)) return FATTN_ERR_MISALIGNED;
+    if (max_seqlen_q > 0x7fffff00) return FATTN_ERR_UNSUPPORTED;
+    DeviceInfo di;
+    st = device_ready(&di);
+    if (st != FATTN_OK) return st;
+    if (!di.fwd_regs_ok) return FATTN_ERR_UNSUPPORTED;
+    const long long BH = static_cast<long long>(nseq) * H;
+    const long long n_qtiles = (max_seqlen_q + 127) / 128;
+    const long long n_pairs = (n_qtiles + 1) / 2;
+    const long long n_items = BH * n_pairs;
+    if (n_items > 0x7fffffffLL) return FATTN_ERR_UNSUPPORTED;
+    CUtensorMap mq, mk, mv;
+    if (encode_map_packed(&mq, q, d, H, total_q) != FATTN_OK || encode_map_packed(&mk, k, d, H, total_k) != FATTN_OK ||
+        encode_map_packed(&mv, v, d, H, total_k) != FATTN_OK)
+        return FATTN_ERR_CUDA;
+    FwdParams p;
+    p.o = o;
+    p.lse = lse;
+    p.visited = visited;
+    p.B = nseq;
+    p.H = H;
+    p.Lq = max_seqlen_q;
+    p.Lk = 0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.window_left = wl < 0 ? -1 : wl;
+    p.window_right = wr < 0 ? -1 : wr;
+    p.n_pairs = static_cast<int>(n_pairs);
+    p.n_items = static_cast<int>(n_items);
+    p.inject_stall = g_inject_stall.exchange(0);
+    p.cu_q = cu_q;
+    p.cu_k = cu_k;
+    p.total_q = total_q;
+    p.total_k = total_k;
+    const int grid = static_cast<int>(n_items < di.num_sms ? n_items : di.num_sms);
+    return launch_prefill_kernel<true>(mq, mk, mv, p, d, grid, static_cast<cudaStream_t>(stream));
 }
 
 int auto_splits(int B, int H, int Lk) {
@@ -201,6 +269,23 @@ int attn_fwd_counted(const void* q, const void* k, const void* v, void* o, float
     if (reinterpret_cast<uintptr_t>(kv_tiles_visited) & 7u) return FATTN_ERR_MISALIGNED;
     return launch_fwd(q, k, v, o, lse, B, H, Lq, Lk, d, scale, causal, window_left, window_right, kv_tiles_visited,
                       stream);
+}
+
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
+                    const int* cu_seqlens_k, int num_seqs, int H, int total_q, int total_k, int max_seqlen_q, int d,
+                    float scale, int causal, int window_left, int window_right, void* stream) {
+    return launch_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, H, total_q, total_k, max_seqlen_q, d,
+                             scale, causal, window_left, window_right, nullptr, stream);
+}
+
+int attn_fwd_varlen_counted(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
+                            const int* cu_seqlens_k, int num_seqs, int H, int total_q, int total_k, int max_seqlen_q,
+                            int d, float scale, int causal, int window_left, int window_right,
+                            unsigned long long* kv_tiles_visited, void* stream) {
+    if (!kv_tiles_visited) return FATTN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(kv_tiles_visited) & 7u) return FATTN_ERR_MISALIGNED;
+    return launch_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, H, total_q, total_k, max_seqlen_q, d,
+                             scale, causal, window_left, window_right, kv_tiles_visited, stream);
 }
 
 int attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int Lq, int Lk,

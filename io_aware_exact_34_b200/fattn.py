@@ -25,6 +25,11 @@ lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i
 lib.attn_fwd.restype = _i
 lib.attn_fwd_counted.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp, _vp]
 lib.attn_fwd_counted.restype = _i
+lib.attn_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp]
+lib.attn_fwd_varlen.restype = _i
+lib.attn_fwd_varlen_counted.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _i,
+                                        _vp, _vp]
+lib.attn_fwd_varlen_counted.restype = _i
 lib.attn_fwd_f32.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp]
 lib.attn_fwd_f32.restype = _i
 lib.attn_decode_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz, _vp]
@@ -114,6 +119,32 @@ def attn_fwd_counted(q, k, v, counter, o=None, lse=None, scale=None, causal=Fals
     _check(lib.attn_fwd_counted(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Lq, Lk, d, scale,
                                 int(bool(causal)), int(window_left), int(window_right), _ptr(counter),
                                 _stream()), "attn_fwd_counted")
+    return o, lse
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, o=None, lse=None, scale=None,
+                    causal=False, window_left=-1, window_right=-1, counter=None):
+    """Packed variable-length prefill.  q: [total_q, H, d], k, v: [total_k, H, d]
+    bf16; cu_seqlens_*: int32 [num_seqs + 1] on the device -> (o, lse [H, total_q])."""
+    _want(q, torch.bfloat16, 3, "q")
+    _want(k, torch.bfloat16, 3, "k")
+    _want(v, torch.bfloat16, 3, "v")
+    _want(cu_seqlens_q, torch.int32, 1, "cu_seqlens_q")
+    _want(cu_seqlens_k, torch.int32, 1, "cu_seqlens_k")
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    nseq = cu_seqlens_q.numel() - 1
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), nseq, H, total_q,
+            total_k, int(max_seqlen_q), d, scale, int(bool(causal)), int(window_left), int(window_right))
+    if counter is None:
+        _check(lib.attn_fwd_varlen(*args, _stream()), "attn_fwd_varlen")
+    else:
+        _check(lib.attn_fwd_varlen_counted(*args, _ptr(counter), _stream()), "attn_fwd_varlen_counted")
     return o, lse
 
 

@@ -118,6 +118,36 @@ def random_qkv(B, H, Lq, Lk, d, dtype="bf16", seed=0, device="cpu"):
     return make_inputs(w, device=device)
 
 
+def varlen_lengths(n_seqs: int, lo: int, hi: int, seed: int):
+    """Sequence lengths drawn uniformly from [lo, hi] (a length mix for packed
+    batches of requests)."""
+    g = torch.Generator().manual_seed(seed)
+    return torch.randint(lo, hi + 1, (n_seqs,), generator=g).tolist()
+
+
+def make_varlen_inputs(lens_q, lens_k, H: int, d: int, seed: int, device="cpu"):
+    """Packed token-major inputs: q [sum(lens_q), H, d], k and v
+    [sum(lens_k), H, d] (bf16, from fp32 N(0, 1) draws, Q then K then V) and
+    the int32 offsets cu_seqlens_q / cu_seqlens_k [n + 1]."""
+    dev = torch.device(device)
+    g = torch.Generator(device=dev.type)
+    g.manual_seed(seed)
+    tq, tk = int(sum(lens_q)), int(sum(lens_k))
+    q = torch.randn((tq, H, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    k = torch.randn((tk, H, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    v = torch.randn((tk, H, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    cu_q = torch.tensor([0] + list(_cumsum(lens_q)), dtype=torch.int32, device=dev)
+    cu_k = torch.tensor([0] + list(_cumsum(lens_k)), dtype=torch.int32, device=dev)
+    return q, k, v, cu_q, cu_k
+
+
+def _cumsum(xs):
+    total = 0
+    for x in xs:
+        total += int(x)
+        yield total
+
+
 def sample_rows(w: Workload, n_random: int, seed: int = 0, full_heads=()):
     """Stratified (b, h, i) row sample: first / last rows, rows at 128-block
     and window edges, plus ``n_random`` uniform rows per head; every row of the

@@ -148,3 +148,20 @@ def test_scheduler_page_example(fl):
     assert (c["visited"], c["partial"]) == (528, 32)
     c = fl.attn_count_blocks(65536, 65536, True, -1, -1, 128, 128)
     assert (c["visited"], c["partial"]) == (131328, 512)
+
+
+def test_varlen_argument_checks(fl):
+    f = fl.lib.attn_fwd_varlen
+    args = lambda **kw: dict(dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, cq=FAKE, ck=FAKE, n=2, H=2, tq=100,
+                                  tk=100, mx=64, d=128, scale=0.1), **kw)
+    def call(**kw):
+        a = args(**kw)
+        return f(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cq"], a["ck"], a["n"], a["H"], a["tq"], a["tk"], a["mx"],
+                 a["d"], a["scale"], 1, -1, -1, None)
+    assert call(cq=None) == fl.FATTN_ERR_INVALID_ARG
+    assert call(n=0) == fl.FATTN_ERR_INVALID_ARG
+    assert call(mx=0) == fl.FATTN_ERR_INVALID_ARG
+    assert call(tq=0) == fl.FATTN_ERR_INVALID_ARG
+    assert call(d=80) == fl.FATTN_ERR_UNSUPPORTED
+    assert call(ck=FAKE + 2) == fl.FATTN_ERR_MISALIGNED
+    assert call(k=FAKE + 8) == fl.FATTN_ERR_MISALIGNED
