@@ -37,6 +37,7 @@ HEADLINE = "causal_4k"
 DECODE = "decode_32k"
 EXTRA = ["window_bidir_32k", "window_causal_32k", "causal_64k_qscale"]
 VARLEN_SEQS, VARLEN_MIN, VARLEN_MAX, VARLEN_H = 32, 256, 4096, 16  # packed batch of causal requests
+PAGE_SIZE = 256  # paged-KV decode: tokens per page
 PREFILL_KERNEL = "attn_fwd_sm100_kernel"
 
 
@@ -359,6 +360,32 @@ def run_ours(args, world, rank, local):
         del dq, dk, dv, do, ws
         torch.cuda.empty_cache()
 
+    # ---------------------------------------------------------------- paged-KV decode
+    decode_paged = None
+    if not args.no_decode and not args.no_extra:
+        wd = synth.WORKLOADS[DECODE]
+        pq, kp, vp, table, seqlens = synth.make_paged_inputs(wd.B, wd.H, wd.Lk, wd.d, PAGE_SIZE,
+                                                             seed=replica_seed(7, rank), device=dev)
+        po = torch.empty_like(pq)
+        pl = torch.empty((wd.B, wd.H), dtype=torch.float32, device=dev)
+        pws = torch.empty(fattn.attn_decode_workspace_bytes(wd.B, wd.H, wd.Lk, wd.d, wd.num_splits),
+                          dtype=torch.uint8, device=dev)
+
+        def pstep():
+            fattn.attn_decode_paged(pq, kp, vp, table, seqlens, o=po, lse=pl, scale=wd.scale,
+                                    num_splits=wd.num_splits, workspace=pws)
+
+        psteps = max(5, min(args.steps, 20))
+        pms = timed(world, pstep, psteps, 3)
+        pbytes = (kp.numel() + vp.numel() + pq.numel() + po.numel()) * 2 + pl.numel() * 4 + table.numel() * 4
+        gbs = pbytes / (pms * 1e-3) / 1e9
+        decode_paged = {"metric": "decode HBM GB/s", "value": world * gbs, "unit": "GB/s", "ms_per_step": pms,
+                        "steps": psteps, "frac_of_hbm_peak": gbs / peaks["hbm_gbs"],
+                        "config": {**wd.describe(), "workload": "decode_32k_paged", "page_size": PAGE_SIZE,
+                                   "layout": "pages [num_pages, page_size, H, d], random block table"}}
+        del pq, kp, vp, table, po, pws
+        torch.cuda.empty_cache()
+
     # ---------------------------------------------------------------- other prefill workloads
     extra = {}
     if not args.no_extra:
@@ -419,7 +446,8 @@ def run_ours(args, world, rank, local):
                            "kv_tiles_visited_per_head": counts["visited"],
                            "kv_tiles_total_per_head": counts["total"]},
                 "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
-                "clocks": clocks, "decode": decode, "extra": extra, "cpu_baseline": cpu}
+                "clocks": clocks, "decode": decode, "decode_paged": decode_paged, "extra": extra,
+                "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)
 
 

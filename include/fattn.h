@@ -158,6 +158,31 @@ int attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
                         int B, int H, int Lk, int d, float scale, int num_splits,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * attn_decode_paged -- attn_decode_splitkv over a paged KV cache ("算子与编译器：
+ * FlashAttention 与长上下文" §5, paged KV cache; the sliding-window prefill
+ * page §7.2 / §8.2): each sequence's keys sit in fixed-size pages of a shared
+ * pool, found through a block table, instead of one contiguous buffer.
+ *
+ *   q            device, bf16 [B,H,1,d]
+ *   k_pages      device, bf16 [num_pages, page_size, H, d] (token-major pages)
+ *   v_pages      device, bf16 [num_pages, page_size, H, d]
+ *   block_table  device, int32 [B, max_pages]: logical page p of sequence b is
+ *                physical page block_table[b*max_pages + p]; indices are
+ *                clamped into [0, num_pages), so no access leaves the pool
+ *   page_size    a power of two >= 16
+ *   seqlens_k    device, int32 [B], required: keys [0, seqlens_k[b]) of
+ *                sequence b are attended (clamped to max_pages*page_size)
+ *   num_splits, workspace, workspace_bytes, o, lse: as attn_decode_splitkv
+ *                with Lk = max_pages * page_size (for the split size and
+ *                attn_decode_workspace_bytes)
+ */
+int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                      const int* block_table, int max_pages, int page_size, int num_pages,
+                      void* o, float* lse, const int* seqlens_k, int B, int H, int d,
+                      float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
 /* Split count attn_decode_splitkv uses for num_splits = 0 (host only). */
 int attn_decode_auto_splits(int B, int H, int Lk, int d);
 

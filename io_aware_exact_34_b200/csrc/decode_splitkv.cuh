@@ -43,13 +43,37 @@ __device__ __forceinline__ void bf16x8_to_float(const uint4& r, float (&f)[8]) {
     }
 }
 
+// Where the key/value rows of one head live.  Contiguous caches: row
+// (b*H + h)*Lk + key of [B, H, Lk, d].  Paged caches ("算子与编译器：
+// FlashAttention 与长上下文" §5, paged KV): logical page key >> page_shift of
+// sequence b is physical page block_table[b][...] of [num_pages, page_size,
+// H, d], and the row is (page * page_size + key % page_size) * H + h.  A page
+// index outside [0, num_pages) is clamped, so a bad table cannot address
+// memory outside the cache.
+struct KvLayout {
+    const int* block_table;  // [B, max_pages] (paged only)
+    int max_pages, page_shift, num_pages;
+};
+
+template <bool kPaged>
+__device__ __forceinline__ long long kv_row(const KvLayout& lay, int b, int h, int H, int Lk, long long key) {
+    if constexpr (kPaged) {
+        int page = __ldg(lay.block_table + static_cast<long long>(b) * lay.max_pages + (key >> lay.page_shift));
+        page = page < 0 ? 0 : (page >= lay.num_pages ? lay.num_pages - 1 : page);
+        const long long tok = (static_cast<long long>(page) << lay.page_shift) | (key & ((1LL << lay.page_shift) - 1));
+        return tok * H + h;
+    } else {
+        return (static_cast<long long>(b) * H + h) * Lk + key;
+    }
+}
+
 // One (split s, head h, batch b) per CTA: partial output and LSE (log2 units).
-template <int D>
+template <int D, bool kPaged>
 __global__ void __launch_bounds__(256)
     decode_split_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                         const __nv_bfloat16* __restrict__ v, const int* __restrict__ seqlens_k,
                         float* __restrict__ ws_o, float* __restrict__ ws_lse, int H, int Lk, int S,
-                        int chunk, float c_log2) {
+                        int chunk, float c_log2, const KvLayout lay) {
     using T = DecodeTraits<D>;
     __shared__ float sm_m[T::G], sm_l[T::G];
     __shared__ float sm_acc[T::G][D];
@@ -77,21 +101,25 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 
-    const __nv_bfloat16* kb = k + bh * static_cast<long long>(Lk) * D + sub * 8;
-    const __nv_bfloat16* vb = v + bh * static_cast<long long>(Lk) * D + sub * 8;
-    for (long long base = k_lo; base < k_hi; base += T::G * T::U) {
-        uint4 kr[T::U], vr[T::U];
+    const __nv_bfloat16* kb = k + sub * 8;
+    const __nv_bfloat16* vb = v + sub * 8;
+    // Rows of one step: keys base + g + u*G, u < U (zeros past the split's end).
+    auto load_step = [&](long long base, uint4 (&kr)[T::U], uint4 (&vr)[T::U]) {
 #pragma unroll
         for (int u = 0; u < T::U; ++u) {
             const long long key = base + g + u * T::G;
             if (key < k_hi) {
-                kr[u] = __ldcs(reinterpret_cast<const uint4*>(kb + key * D));
-                vr[u] = __ldcs(reinterpret_cast<const uint4*>(vb + key * D));
+                const long long row = kv_row<kPaged>(lay, b, h, H, Lk, key);
+                kr[u] = __ldcs(reinterpret_cast<const uint4*>(kb + row * D));
+                vr[u] = __ldcs(reinterpret_cast<const uint4*>(vb + row * D));
             } else {
                 kr[u] = make_uint4(0u, 0u, 0u, 0u);
                 vr[u] = make_uint4(0u, 0u, 0u, 0u);
             }
         }
+    };
+    // Online-softmax update of this group's (m, l, acc) with one step of rows.
+    auto consume_step = [&](long long base, const uint4 (&kr)[T::U], const uint4 (&vr)[T::U]) {
         float x[T::U];
 #pragma unroll
         for (int u = 0; u < T::U; ++u) {
@@ -123,6 +151,27 @@ __global__ void __launch_bounds__(256)
             for (int e = 0; e < 8; ++e) acc[e] = fmaf(pu, vf[e], acc[e]);
         }
         m = m_new;
+    };
+    constexpr long long STEP = T::G * T::U;
+    if constexpr (kPaged) {
+        // Paged rows: each row address waits on a block-table load; measured
+        // on B200 this variant streams faster without the explicit pipeline.
+        uint4 kA[T::U], vA[T::U];
+        for (long long base = k_lo; base < k_hi; base += STEP) {
+            load_step(base, kA, vA);
+            consume_step(base, kA, vA);
+        }
+    } else {
+        // Software pipeline: the next step's rows are in flight while this
+        // step's are reduced (steps past the split's end load nothing, weigh 0).
+        uint4 kA[T::U], vA[T::U], kB[T::U], vB[T::U];
+        load_step(k_lo, kA, vA);
+        for (long long base = k_lo; base < k_hi; base += 2 * STEP) {
+            load_step(base + STEP, kB, vB);
+            consume_step(base, kA, vA);
+            load_step(base + 2 * STEP, kA, vA);
+            consume_step(base + STEP, kB, vB);
+        }
     }
 
     if (sub == 0) {

@@ -349,11 +349,59 @@ int attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
     const auto* kb = static_cast<const __nv_bfloat16*>(k_cache);
     const auto* vb = static_cast<const __nv_bfloat16*>(v_cache);
     auto* ob = static_cast<__nv_bfloat16*>(o);
+    const KvLayout lay{nullptr, 0, 0, 0};
     if (d == 128) {
-        decode_split_kernel<128><<<grid, 256, 0, s>>>(qb, kb, vb, seqlens_k, ws_o, ws_lse, H, Lk, S, chunk, c_log2);
+        decode_split_kernel<128, false><<<grid, 256, 0, s>>>(qb, kb, vb, seqlens_k, ws_o, ws_lse, H, Lk, S, chunk, c_log2, lay);
         decode_merge_kernel<128><<<B * H, 128, 0, s>>>(ws_o, ws_lse, ob, lse, S);
     } else {
-        decode_split_kernel<64><<<grid, 256, 0, s>>>(qb, kb, vb, seqlens_k, ws_o, ws_lse, H, Lk, S, chunk, c_log2);
+        decode_split_kernel<64, false><<<grid, 256, 0, s>>>(qb, kb, vb, seqlens_k, ws_o, ws_lse, H, Lk, S, chunk, c_log2, lay);
+        decode_merge_kernel<64><<<B * H, 64, 0, s>>>(ws_o, ws_lse, ob, lse, S);
+    }
+    return cudaGetLastError() == cudaSuccess ? FATTN_OK : FATTN_ERR_CUDA;
+}
+
+int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int* block_table, int max_pages,
+                      int page_size, int num_pages, void* o, float* lse, const int* seqlens_k, int B, int H, int d,
+                      float scale, int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!q || !k_pages || !v_pages || !block_table || !seqlens_k || !o) return FATTN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || max_pages < 1 || num_pages < 1 || num_splits < 0) return FATTN_ERR_INVALID_ARG;
+    if (page_size < 16 || (page_size & (page_size - 1)) != 0) return FATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return FATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FATTN_ERR_UNSUPPORTED;
+    const long long max_len = static_cast<long long>(max_pages) * page_size;
+    if (B > 65535 || H > 65535 || max_len > 0x7fffff00 || static_cast<long long>(num_pages) * page_size > (1LL << 40))
+        return FATTN_ERR_UNSUPPORTED;
+    const int Lk = static_cast<int>(max_len);
+    const int S = num_splits == 0 ? auto_splits(B, H, Lk) : num_splits;
+    if (S > Lk) return FATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o)) return FATTN_ERR_MISALIGNED;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FATTN_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(seqlens_k) & 3u) || (reinterpret_cast<uintptr_t>(block_table) & 3u))
+        return FATTN_ERR_MISALIGNED;
+    const size_t need = attn_decode_workspace_bytes(B, H, Lk, d, S);
+    if (!workspace || workspace_bytes < need) return FATTN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FATTN_ERR_MISALIGNED;
+    DeviceInfo di;
+    int st = device_ready(&di);
+    if (st != FATTN_OK) return st;
+    float* ws_o = static_cast<float*>(workspace);
+    float* ws_lse = ws_o + static_cast<size_t>(B) * H * S * d;
+    const int chunk = static_cast<int>((static_cast<long long>(Lk) + S - 1) / S);
+    const float c_log2 = scale * 1.4426950408889634f;
+    int shift = 0;
+    while ((1 << shift) < page_size) ++shift;
+    const KvLayout lay{block_table, max_pages, shift, num_pages};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    dim3 grid(S, H, B);
+    const auto* qb = static_cast<const __nv_bfloat16*>(q);
+    const auto* kb = static_cast<const __nv_bfloat16*>(k_pages);
+    const auto* vb = static_cast<const __nv_bfloat16*>(v_pages);
+    auto* ob = static_cast<__nv_bfloat16*>(o);
+    if (d == 128) {
+        decode_split_kernel<128, true><<<grid, 256, 0, s>>>(qb, kb, vb, seqlens_k, ws_o, ws_lse, H, Lk, S, chunk, c_log2, lay);
+        decode_merge_kernel<128><<<B * H, 128, 0, s>>>(ws_o, ws_lse, ob, lse, S);
+    } else {
+        decode_split_kernel<64, true><<<grid, 256, 0, s>>>(qb, kb, vb, seqlens_k, ws_o, ws_lse, H, Lk, S, chunk, c_log2, lay);
         decode_merge_kernel<64><<<B * H, 64, 0, s>>>(ws_o, ws_lse, ob, lse, S);
     }
     return cudaGetLastError() == cudaSuccess ? FATTN_OK : FATTN_ERR_CUDA;

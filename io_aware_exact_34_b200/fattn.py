@@ -36,6 +36,8 @@ lib.attn_decode_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i
 lib.attn_decode_splitkv.restype = _i
 lib.attn_decode_splitkv_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp]
 lib.attn_decode_splitkv_noalloc.restype = _i
+lib.attn_decode_paged.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp, _sz, _vp]
+lib.attn_decode_paged.restype = _i
 lib.attn_decode_auto_splits.argtypes = [_i, _i, _i, _i]
 lib.attn_decode_auto_splits.restype = _i
 lib.attn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
@@ -219,6 +221,34 @@ def attn_decode_splitkv_noalloc(q, k_cache, v_cache, o=None, lse=None, seqlens_k
     _check(lib.attn_decode_splitkv_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
                                            _ptr(seqlens_k), B, H, Lk, d, scale, int(num_splits), _stream()),
            "attn_decode_splitkv_noalloc")
+    return o, lse
+
+
+def attn_decode_paged(q, k_pages, v_pages, block_table, seqlens_k, o=None, lse=None, scale=None, num_splits=0,
+                      workspace=None):
+    """Split-KV decode over a paged cache.  q: [B,H,1,d]; k_pages, v_pages:
+    [num_pages, page_size, H, d] bf16; block_table: int32 [B, max_pages];
+    seqlens_k: int32 [B] -> (o [B,H,1,d], lse [B,H])."""
+    _want(q, torch.bfloat16, 4, "q")
+    _want(k_pages, torch.bfloat16, 4, "k_pages")
+    _want(v_pages, torch.bfloat16, 4, "v_pages")
+    _want(block_table, torch.int32, 2, "block_table")
+    _want(seqlens_k, torch.int32, 1, "seqlens_k")
+    B, H, _, d = q.shape
+    num_pages, page_size = k_pages.shape[0], k_pages.shape[1]
+    max_pages = block_table.shape[1]
+    Lk = max_pages * page_size
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    S = num_splits if num_splits > 0 else attn_decode_auto_splits(B, H, Lk, d)
+    if workspace is None:
+        workspace = torch.empty(attn_decode_workspace_bytes(B, H, Lk, d, S), dtype=torch.uint8, device=q.device)
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    _check(lib.attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), max_pages, page_size,
+                                 num_pages, _ptr(o), _ptr(lse), _ptr(seqlens_k), B, H, d, scale, S, _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream()), "attn_decode_paged")
     return o, lse
 
 

@@ -148,6 +148,47 @@ def _cumsum(xs):
         yield total
 
 
+def scatter_to_pages(k, v, page_size: int, seed: int, extra_pages: int = 0):
+    """Place a contiguous cache k, v [B, H, L, d] (L a multiple of page_size)
+    into a pool of pages [num_pages, page_size, H, d] in a seeded random page
+    order; returns (k_pages, v_pages, block_table int32 [B, L / page_size]).
+    extra_pages unused pages are added to the pool.  Pure data movement."""
+    B, H, L, d = k.shape
+    assert L % page_size == 0
+    per_seq = L // page_size
+    num_pages = B * per_seq + extra_pages
+    g = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(num_pages, generator=g)[: B * per_seq].view(B, per_seq)
+    kp = torch.zeros((num_pages, page_size, H, d), dtype=k.dtype, device=k.device)
+    vp = torch.zeros_like(kp)
+    # [B, H, per_seq, page_size, d] -> [B, per_seq, page_size, H, d]
+    kk = k.view(B, H, per_seq, page_size, d).permute(0, 2, 3, 1, 4)
+    vv = v.view(B, H, per_seq, page_size, d).permute(0, 2, 3, 1, 4)
+    idx = perm.to(k.device).reshape(-1)
+    kp[idx] = kk.reshape(B * per_seq, page_size, H, d)
+    vp[idx] = vv.reshape(B * per_seq, page_size, H, d)
+    return kp, vp, perm.to(torch.int32).to(k.device).contiguous()
+
+
+def make_paged_inputs(B: int, H: int, L: int, d: int, page_size: int, seed: int, device="cuda"):
+    """A decode batch over a paged cache: q [B, H, 1, d], page pools
+    [B * L / page_size, page_size, H, d] drawn directly (fp32 N(0, 1) rounded
+    to bf16, pool by pool), a seeded random block table [B, L / page_size]
+    (a permutation of the pool) and full lengths L."""
+    dev = torch.device(device)
+    g = torch.Generator(device=dev.type)
+    g.manual_seed(seed)
+    per_seq = L // page_size
+    num_pages = B * per_seq
+    q = torch.randn((B, H, 1, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    kp = _draw((num_pages, page_size, H, d), g, dev, torch.bfloat16)
+    vp = _draw((num_pages, page_size, H, d), g, dev, torch.bfloat16)
+    gc = torch.Generator().manual_seed(seed)
+    table = torch.randperm(num_pages, generator=gc).view(B, per_seq).to(torch.int32).to(dev)
+    seqlens = torch.full((B,), L, dtype=torch.int32, device=dev)
+    return q, kp, vp, table, seqlens
+
+
 def sample_rows(w: Workload, n_random: int, seed: int = 0, full_heads=()):
     """Stratified (b, h, i) row sample: first / last rows, rows at 128-block
     and window edges, plus ``n_random`` uniform rows per head; every row of the

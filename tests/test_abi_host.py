@@ -165,3 +165,16 @@ def test_varlen_argument_checks(fl):
     assert call(d=80) == fl.FATTN_ERR_UNSUPPORTED
     assert call(ck=FAKE + 2) == fl.FATTN_ERR_MISALIGNED
     assert call(k=FAKE + 8) == fl.FATTN_ERR_MISALIGNED
+
+
+def test_paged_decode_argument_checks(fl):
+    def call(page=16, table=FAKE, sl=FAKE, ws=FAKE, ws_bytes=1 << 20, d=128, S=1):
+        return fl.lib.attn_decode_paged(FAKE, FAKE, FAKE, table, 4, page, 4, FAKE, None, sl, 1, 1, d, 0.1, S, ws,
+                                        ws_bytes, None)
+    assert call(page=24) == fl.FATTN_ERR_INVALID_ARG      # not a power of two
+    assert call(page=8) == fl.FATTN_ERR_INVALID_ARG       # below 16
+    assert call(table=None) == fl.FATTN_ERR_INVALID_ARG
+    assert call(sl=None) == fl.FATTN_ERR_INVALID_ARG      # lengths are required
+    assert call(d=96) == fl.FATTN_ERR_UNSUPPORTED
+    assert call(table=FAKE + 2) == fl.FATTN_ERR_MISALIGNED
+    assert call(ws=None) == fl.FATTN_ERR_WORKSPACE
