@@ -373,6 +373,99 @@ void oracle_decode_splitmerge(const void* q, const void* k, const void* v, int d
 }
 
 /*
+ * Gradients of exact attention ([P2] §3.3: the backward pass recomputes the
+ * scores instead of storing them).  With the loss L = sum_i dO_i . O_i, by the
+ * chain rule through O_i = sum_j P_ij v_j and the row softmax P_ij:
+ *   dV_j  = sum_i P_ij dO_i
+ *   dP_ij = dO_i . v_j
+ *   D_i   = sum_j P_ij dP_ij  (= dO_i . O_i)
+ *   dS_ij = P_ij (dP_ij - D_i)
+ *   dQ_i  = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i
+ * All in fp64 from the widened inputs; P by the definition (masked entries 0,
+ * rows without an allowed key contribute nothing).  do_ has q's layout.
+ */
+void oracle_attn_bwd(const void* q, const void* k, const void* v, const void* do_, int dtype,
+                     double* dq, double* dk, double* dv, int B, int H, int Lq, int Lk, int d,
+                     double scale, int causal, int wl, int wr) {
+    std::vector<double> Qd(static_cast<size_t>(Lq) * d), Kd(static_cast<size_t>(Lk) * d),
+        Vd(static_cast<size_t>(Lk) * d), Od(static_cast<size_t>(Lq) * d);
+    std::vector<double> P(static_cast<size_t>(Lq) * Lk);
+    for (long long bh = 0; bh < static_cast<long long>(B) * H; ++bh) {
+        widen_block(q, bh * Lq * d, static_cast<long long>(Lq) * d, dtype, Qd.data());
+        widen_block(do_, bh * Lq * d, static_cast<long long>(Lq) * d, dtype, Od.data());
+        widen_block(k, bh * Lk * d, static_cast<long long>(Lk) * d, dtype, Kd.data());
+        widen_block(v, bh * Lk * d, static_cast<long long>(Lk) * d, dtype, Vd.data());
+        double* dq_h = dq + bh * Lq * d;
+        double* dk_h = dk + bh * Lk * d;
+        double* dv_h = dv + bh * Lk * d;
+        /* probabilities and the row gradients, row by row */
+#pragma omp parallel for schedule(dynamic, 4)
+        for (long long i = 0; i < Lq; ++i) {
+            double* Pi = P.data() + i * Lk;
+            double M = NEG_INF;
+            for (long long j = 0; j < Lk; ++j) {
+                if (!allowed(i, j, Lq, Lk, Lk, causal, wl, wr)) { Pi[j] = NEG_INF; continue; }
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) dot += Qd[i * d + c] * Kd[j * d + c];
+                Pi[j] = scale * dot;
+                if (Pi[j] > M) M = Pi[j];
+            }
+            double Z = 0.0;
+            for (long long j = 0; j < Lk; ++j) {
+                Pi[j] = (M == NEG_INF || Pi[j] == NEG_INF) ? 0.0 : std::exp(Pi[j] - M);
+                Z += Pi[j];
+            }
+            for (long long j = 0; j < Lk; ++j) Pi[j] = Z > 0.0 ? Pi[j] / Z : 0.0;
+            /* D_i = sum_j P_ij dP_ij, then dQ_i = scale sum_j dS_ij k_j */
+            double Di = 0.0;
+            for (long long j = 0; j < Lk; ++j) {
+                if (Pi[j] == 0.0) continue;
+                double dp = 0.0;
+                for (int c = 0; c < d; ++c) dp += Od[i * d + c] * Vd[j * d + c];
+                Di += Pi[j] * dp;
+            }
+            for (int c = 0; c < d; ++c) dq_h[i * d + c] = 0.0;
+            for (long long j = 0; j < Lk; ++j) {
+                if (Pi[j] == 0.0) continue;
+                double dp = 0.0;
+                for (int c = 0; c < d; ++c) dp += Od[i * d + c] * Vd[j * d + c];
+                const double ds = Pi[j] * (dp - Di);
+                for (int c = 0; c < d; ++c) dq_h[i * d + c] += scale * ds * Kd[j * d + c];
+            }
+        }
+        /* column gradients dK_j, dV_j need every row's D_i: recompute per column */
+        std::vector<double> D(Lq);
+#pragma omp parallel for schedule(dynamic, 4)
+        for (long long i = 0; i < Lq; ++i) {
+            const double* Pi = P.data() + i * Lk;
+            double Di = 0.0;
+            for (long long j = 0; j < Lk; ++j) {
+                if (Pi[j] == 0.0) continue;
+                double dp = 0.0;
+                for (int c = 0; c < d; ++c) dp += Od[i * d + c] * Vd[j * d + c];
+                Di += Pi[j] * dp;
+            }
+            D[i] = Di;
+        }
+#pragma omp parallel for schedule(dynamic, 4)
+        for (long long j = 0; j < Lk; ++j) {
+            for (int c = 0; c < d; ++c) { dk_h[j * d + c] = 0.0; dv_h[j * d + c] = 0.0; }
+            for (long long i = 0; i < Lq; ++i) {
+                const double Pij = P[i * Lk + j];
+                if (Pij == 0.0) continue;
+                double dp = 0.0;
+                for (int c = 0; c < d; ++c) dp += Od[i * d + c] * Vd[j * d + c];
+                const double ds = Pij * (dp - D[i]);
+                for (int c = 0; c < d; ++c) {
+                    dv_h[j * d + c] += Pij * Od[i * d + c];
+                    dk_h[j * d + c] += scale * ds * Qd[i * d + c];
+                }
+            }
+        }
+    }
+}
+
+/*
  * Brute-force enumeration of the mask ([P2] §5.4 block-pair accounting): for
  * block_q x block_k tiles of the Lq x Lk score matrix (rows i < Lq only),
  *   pairs   = number of allowed (i, j),

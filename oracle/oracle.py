@@ -51,6 +51,7 @@ def _load():
             lib.oracle_attn_tiled.argtypes = [vp, vp, vp, i, dp, dp, i, i, i, i, i, d, i, i, i, i, i, i, i, llp]
             lib.oracle_decode_splitmerge.argtypes = [vp, vp, vp, i, dp, dp, i, i, i, i, d, ip, i]
             lib.oracle_count_blocks.argtypes = [i, i, i, i, i, i, i, llp, llp, llp, llp]
+            lib.oracle_attn_bwd.argtypes = [vp, vp, vp, vp, i, dp, dp, dp, i, i, i, i, i, d, i, i, i]
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_set_num_threads.argtypes = [i]
             _lib = lib
@@ -194,6 +195,21 @@ def decode_splitmerge(q, k, v, scale, num_splits, seqlens_k=None):
                                      B, H, Lk, d, float(scale), sl, int(num_splits))
     del keep
     return o, lse
+
+
+def attn_bwd(q, k, v, do, scale, causal=False, window_left=-1, window_right=-1):
+    """Gradients (dQ, dK, dV) of L = sum(dO * O) for exact masked attention,
+    fp64.  q, do: [B,H,Lq,d]; k, v: [B,H,Lk,d]."""
+    (qa, ka, va, da), dt = _same_kind(q, k, v, do)
+    B, H, Lq, d = qa.shape
+    Lk = ka.shape[2]
+    dq = np.empty((B, H, Lq, d), np.float64)
+    dk = np.empty((B, H, Lk, d), np.float64)
+    dv = np.empty((B, H, Lk, d), np.float64)
+    _load().oracle_attn_bwd(_ptr(qa), _ptr(ka), _ptr(va), _ptr(da), dt, _dptr(dq), _dptr(dk), _dptr(dv),
+                            B, H, Lq, Lk, d, float(scale), int(bool(causal)), int(window_left),
+                            int(window_right))
+    return dq, dk, dv
 
 
 def count_blocks(Lq, Lk, causal, window_left, window_right, block_q, block_k):
