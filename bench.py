@@ -7,10 +7,10 @@ A step is one pass of the prefill hot path (closed-form KV tile ranges, TMA
 Q/K/V tiles, tcgen05 S = Q K^T, masked exp2 online softmax, P V, O / l and
 LSE) over the causal 4 x 16 x 4096, d = 128 bf16 workload; ``value`` is its
 in-mask TFLOP/s (4 d FLOPs per allowed (q, k) pair per head) with inputs
-resident in HBM.  The same run times the split-KV decode path (split kernel +
-LSE merge) on the 64 x 32 x 32768 cache and reports it under ``decode`` in
-GB/s of K/V/q/o/lse traffic, and the sliding-window / long-causal prefill
-workloads under ``extra``.
+resident in HBM.  The same run times the backward with recomputation on that
+workload (``bwd``), the split-KV decode path (split kernel + LSE merge) on the
+64 x 32 x 32768 cache under ``decode`` in GB/s of K/V/q/o/lse traffic, and the
+sliding-window / long-causal prefill workloads under ``extra``.
 
 Multi-GPU (torchrun, one rank per GPU): (batch, head) units are independent,
 so every rank runs its own full copy of the workload with no collective on the
@@ -330,6 +330,33 @@ def run_ours(args, world, rank, local):
                "d2h_bytes_per_step": int(o.numel() * o.element_size() + lse.numel() * 4)}
         del qh, kh, vh, oh, lh, qd, kd, vd
 
+    # ---------------------------------------------------------------- backward (recomputation)
+    bwd = None
+    if not args.no_bwd:
+        step()  # O and LSE of the forward, the backward's inputs
+        dout = synth.random_dout(w.B, w.H, w.Lq, w.d, "bf16", seed=replica_seed(w.seed, rank), device=dev)
+        gq, gk, gv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        gws = torch.empty(fattn.attn_bwd_workspace_bytes(w.B, w.H, w.Lq, w.d), dtype=torch.uint8, device=dev)
+
+        def bstep():
+            fattn.attn_bwd(q, k, v, o, dout, lse, scale=w.scale, causal=w.causal, window_left=w.window_left,
+                           window_right=w.window_right, dq=gq, dk=gk, dv=gv, workspace=gws)
+
+        bsteps = max(3, min(args.steps, 20))
+        bms = timed(world, bstep, bsteps, 3)
+        bflops = 2.5 * flops  # five products per allowed pair instead of two
+        tf = bflops / (bms * 1e-3) / 1e12
+        bwd = {"metric": "attention bwd TFLOP/s (in-mask FLOPs: 10 d per allowed pair)", "value": world * tf,
+               "unit": "TFLOP/s", "ms_per_step": bms, "steps": bsteps,
+               "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                            "frac": tf / peaks["bf16_tflops"], "traffic": None,
+                            "peak_source": f"{peak_src} bf16 dense (burst)",
+                            "kernels": ["bwd_prep_kernel", "attn_bwd_sm100_kernel", "bwd_dq_kernel"]},
+               "config": {**w.describe(), "pass": "backward with recomputation from LSE"},
+               "gpu_launches": 3 * bsteps}
+        del dout, gq, gk, gv, gws
+        torch.cuda.empty_cache()
+
     # ---------------------------------------------------------------- decode
     decode = None
     if not args.no_decode:
@@ -446,7 +473,7 @@ def run_ours(args, world, rank, local):
                            "kv_tiles_visited_per_head": counts["visited"],
                            "kv_tiles_total_per_head": counts["total"]},
                 "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
-                "clocks": clocks, "decode": decode, "decode_paged": decode_paged, "extra": extra,
+                "clocks": clocks, "bwd": bwd, "decode": decode, "decode_paged": decode_paged, "extra": extra,
                 "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)
 
@@ -462,6 +489,7 @@ def main():
     ap.add_argument("--no-clocks", action="store_true", help="no nvidia-smi sampling or soak (profiling runs)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -205,13 +205,71 @@ int attn_count_blocks(int Lq, int Lk, int causal, int window_left, int window_ri
                       int block_q, int block_k, long long* visited, long long* total,
                       long long* partial, long long* pairs);
 
+/*
+ * attn_bwd -- bf16 backward of attn_fwd with recomputation: the score tiles
+ * are rebuilt from Q, K and the forward's LSE instead of being stored (the
+ * sliding-window FlashAttention prefill page §3.3; the bomianfm.com
+ * FlashAttention answer, "recomputation" bullet).  The gradients of
+ * L = sum(dO * O) through the forward above, with P = exp(scale Q K^T - LSE)
+ * on allowed pairs and 0 elsewhere:
+ *
+ *     dV = P^T dO,  dP = dO V^T,  D_i = dO_i . O_i,  dS = P o (dP - D),
+ *     dQ = scale dS K,  dK = scale dS^T Q
+ *
+ *   q, k, v   device, bf16, as passed to attn_fwd
+ *   o         device, bf16 [B,H,Lq,d]: attn_fwd's output for these inputs
+ *   dout      device, bf16 [B,H,Lq,d]: dL/dO
+ *   lse       device, fp32 [B,H,Lq]: attn_fwd's LSE for these inputs (rows
+ *             without keys hold -inf and get zero gradient)
+ *   dq        device, bf16 [B,H,Lq,d] (written)
+ *   dk, dv    device, bf16 [B,H,Lk,d] (written; keys no query sees get 0)
+ *   B, H, Lq, Lk, d, scale, causal, window_left, window_right: as attn_fwd
+ *   workspace device scratch of at least attn_bwd_workspace_bytes(B,H,Lq,d)
+ *             bytes, 16-byte aligned; contents on entry are ignored and on
+ *             return unspecified (it holds the fp32 dQ accumulator)
+ * Every tensor is 16-byte aligned (lse 4-byte).  Three kernels are enqueued
+ * on `stream`: the D_i / LSE pre-pass, the main kernel (one CTA per 128-key
+ * tile per head, tensor cores) and the dQ conversion.
+ *
+ * Precision: products in bf16 with fp32 accumulation; P and dS are rounded to
+ * bf16 before they enter a product, dS is formed from the bf16 P; dQ is
+ * accumulated in fp32 across KV tiles (atomic adds, so its summation order
+ * varies between runs); outputs are rounded to bf16 once.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv,
+             int B, int H, int Lq, int Lk, int d, float scale,
+             int causal, int window_left, int window_right,
+             void* workspace, size_t workspace_bytes, void* stream);
+
+/* attn_bwd that also adds, to *q_tiles_visited (device, unsigned 64-bit,
+ * caller-zeroed), the number of (128-key tile, 128-query tile) pairs the main
+ * kernel computed; it equals attn_bwd_count_blocks(..., 128, 128) times B*H. */
+int attn_bwd_counted(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv,
+                     int B, int H, int Lq, int Lk, int d, float scale,
+                     int causal, int window_left, int window_right,
+                     void* workspace, size_t workspace_bytes,
+                     unsigned long long* q_tiles_visited, void* stream);
+
+/* Bytes of workspace attn_bwd needs: B*H*Lq_pad*(d+2)*4 with Lq_pad = Lq
+ * rounded up to 128.  0 on invalid input.  Host only. */
+size_t attn_bwd_workspace_bytes(int B, int H, int Lq, int d);
+
+/* Host-only: the number of (block_q query tile, block_k key tile) pairs the
+ * backward's schedule visits for one head, summed over the key tiles (each
+ * key tile walks the query tiles of the band in closed form).  It equals
+ * attn_count_blocks's `visited`: both are the tiles with an allowed pair. */
+int attn_bwd_count_blocks(int Lq, int Lk, int causal, int window_left, int window_right,
+                          int block_q, int block_k, long long* visited);
+
 /* Human-readable name of a fattn_status value. */
 const char* fattn_status_string(int status);
 
 /*
  * fattn_device_status -- synchronises `stream`, then returns and clears the
  * device status word of the current device (FATTN_OK, or FATTN_ERR_TIMEOUT if
- * a bounded wait in a prefill kernel expired since the last call).  A debugging
+ * a bounded wait in a prefill or backward kernel expired since the last call).  A debugging
  * aid; it blocks the calling thread.
  */
 int fattn_device_status(void* stream);

@@ -174,10 +174,6 @@ struct RowPlan {
     bool tile_exists, valid;
 };
 
-__device__ __forceinline__ int clamp_int(long long x) {
-    return static_cast<int>(x < -(1LL << 30) ? -(1LL << 30) : (x > (1LL << 30) ? (1LL << 30) : x));
-}
-
 template <int D, bool kVarlen>
 __device__ __forceinline__ RowPlan row_plan(const FwdParams& p, int item, int t, int row) {
     RowPlan rp;

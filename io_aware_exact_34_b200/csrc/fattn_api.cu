@@ -14,6 +14,7 @@
 
 #include "fattn.h"
 
+#include "attn_bwd_sm100.cuh"
 #include "attn_fwd_f32.cuh"
 #include "attn_fwd_sm100.cuh"
 #include "decode_splitkv.cuh"
@@ -87,6 +88,8 @@ int device_ready(DeviceInfo* out) {
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64>::SMEM_BYTES);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_bwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdTraits<128>::SMEM_BYTES);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_bwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdTraits<64>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, F32Traits<128>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, F32Traits<64>::SMEM_BYTES);
             if (e != cudaSuccess) {
@@ -242,6 +245,92 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
     p.total_k = total_k;
     const int grid = static_cast<int>(n_items < di.num_sms ? n_items : di.num_sms);
     return launch_prefill_kernel<true>(mq, mk, mv, p, d, grid, static_cast<cudaStream_t>(stream));
+}
+
+long long bwd_lq_pad(int Lq) { return (static_cast<long long>(Lq) + 127) / 128 * 128; }
+
+// Q tiles visited by all KV tiles of one head: the backward's work count.
+long long bwd_visited_tiles(const Band& band, int Lk, int bq, int bk) {
+    long long n = 0;
+    for (long long k0 = 0; k0 < Lk; k0 += bk) {
+        const long long k_last = k0 + bk - 1 < Lk - 1 ? k0 + bk - 1 : Lk - 1;
+        int lo = 0, hi = 0;
+        q_tile_range(band, k0, k_last, bq, &lo, &hi);
+        n += hi - lo;
+    }
+    return n;
+}
+
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
+               void* dk, void* dv, int B, int H, int Lq, int Lk, int d, float scale, int causal, int wl, int wr,
+               void* workspace, size_t workspace_bytes, unsigned long long* visited, void* stream) {
+    if (!dout || !lse || !dq || !dk || !dv) return FATTN_ERR_INVALID_ARG;
+    int st = check_prefill(q, k, v, o, lse, B, H, Lq, Lk, d, scale);
+    if (st != FATTN_OK) return st;
+    if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return FATTN_ERR_MISALIGNED;
+    const long long BH = static_cast<long long>(B) * H;
+    const long long n_kv = (Lk + 127) / 128;
+    if (BH * n_kv > 0x7fffffffLL) return FATTN_ERR_UNSUPPORTED;
+    const size_t need = attn_bwd_workspace_bytes(B, H, Lq, d);
+    if (!workspace || workspace_bytes < need) return FATTN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FATTN_ERR_MISALIGNED;
+    DeviceInfo di;
+    st = device_ready(&di);
+    if (st != FATTN_OK) return st;
+    const long long Lq_pad = bwd_lq_pad(Lq);
+    CUtensorMap mq, mk, mv, mdo;
+    if (encode_map(&mq, q, d, Lq, BH) != FATTN_OK || encode_map(&mk, k, d, Lk, BH) != FATTN_OK ||
+        encode_map(&mv, v, d, Lk, BH) != FATTN_OK || encode_map(&mdo, dout, d, Lq, BH) != FATTN_OK)
+        return FATTN_ERR_CUDA;
+    float* lse2 = static_cast<float*>(workspace);
+    float* dsum = lse2 + BH * Lq_pad;
+    float* dq_acc = dsum + BH * Lq_pad;
+    const Band band = make_band(Lq, Lk, causal, wl, wr);
+    BwdParams p;
+    p.lse2 = lse2;
+    p.dsum = dsum;
+    p.dq_acc = dq_acc;
+    p.dk = dk;
+    p.dv = dv;
+    p.visited = visited;
+    p.BH = static_cast<int>(BH);
+    p.Lq = Lq;
+    p.Lk = Lk;
+    p.Lq_pad = static_cast<int>(Lq_pad);
+    p.n_kv = static_cast<int>(n_kv);
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.window_left = wl < 0 ? -1 : wl;
+    p.window_right = wr < 0 ? -1 : wr;
+    {
+        // longest KV tiles first: compare the Q ranges of the first and last KV tile
+        int lo0 = 0, hi0 = 0, lo1 = 0, hi1 = 0;
+        const long long last0 = (n_kv - 1) * 128;
+        q_tile_range(band, 0, 127 < Lk - 1 ? 127 : Lk - 1, 128, &lo0, &hi0);
+        q_tile_range(band, last0, Lk - 1, 128, &lo1, &hi1);
+        p.reverse = (hi1 - lo1) > (hi0 - lo0) ? 1 : 0;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const auto* ob = static_cast<const __nv_bfloat16*>(o);
+    const auto* dob = static_cast<const __nv_bfloat16*>(dout);
+    auto* dqb = static_cast<__nv_bfloat16*>(dq);
+    const long long prep_threads = BH * Lq_pad * (d / 8);
+    const long long fin_threads = BH * Lq * (d / 8);
+    if ((prep_threads + 255) / 256 > 0x7fffffffLL) return FATTN_ERR_UNSUPPORTED;
+    const unsigned prep_grid = static_cast<unsigned>((prep_threads + 255) / 256);
+    const unsigned fin_grid = static_cast<unsigned>((fin_threads + 255) / 256);
+    const unsigned grid = static_cast<unsigned>(BH * n_kv);
+    if (d == 128) {
+        bwd_prep_kernel<128><<<prep_grid, 256, 0, s>>>(ob, dob, lse, lse2, dsum, dq_acc, p.BH, Lq, p.Lq_pad);
+        attn_bwd_sm100_kernel<128><<<grid, BwdTraits<128>::THREADS, BwdTraits<128>::SMEM_BYTES, s>>>(mq, mk, mv, mdo, p);
+        bwd_dq_kernel<128><<<fin_grid, 256, 0, s>>>(dq_acc, dqb, p.BH, Lq, p.Lq_pad, scale);
+    } else {
+        bwd_prep_kernel<64><<<prep_grid, 256, 0, s>>>(ob, dob, lse, lse2, dsum, dq_acc, p.BH, Lq, p.Lq_pad);
+        attn_bwd_sm100_kernel<64><<<grid, BwdTraits<64>::THREADS, BwdTraits<64>::SMEM_BYTES, s>>>(mq, mk, mv, mdo, p);
+        bwd_dq_kernel<64><<<fin_grid, 256, 0, s>>>(dq_acc, dqb, p.BH, Lq, p.Lq_pad, scale);
+    }
+    return cudaGetLastError() == cudaSuccess ? FATTN_OK : FATTN_ERR_CUDA;
 }
 
 int auto_splits(int B, int H, int Lk) {
@@ -431,6 +520,36 @@ int attn_count_blocks(int Lq, int Lk, int causal, int window_left, int window_ri
     if (total) *total = nq * nk;
     if (partial) *partial = n_partial;
     if (pairs) *pairs = n_pairs;
+    return FATTN_OK;
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int Lq, int d) {
+    if (B < 1 || H < 1 || Lq < 1 || (d != 64 && d != 128)) return 0;
+    return static_cast<size_t>(B) * H * static_cast<size_t>(bwd_lq_pad(Lq)) * (static_cast<size_t>(d) + 2) * sizeof(float);
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
+             void* dk, void* dv, int B, int H, int Lq, int Lk, int d, float scale, int causal, int window_left,
+             int window_right, void* workspace, size_t workspace_bytes, void* stream) {
+    return launch_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, Lq, Lk, d, scale, causal, window_left, window_right,
+                      workspace, workspace_bytes, nullptr, stream);
+}
+
+int attn_bwd_counted(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                     void* dq, void* dk, void* dv, int B, int H, int Lq, int Lk, int d, float scale, int causal,
+                     int window_left, int window_right, void* workspace, size_t workspace_bytes,
+                     unsigned long long* q_tiles_visited, void* stream) {
+    if (!q_tiles_visited) return FATTN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(q_tiles_visited) & 7u) return FATTN_ERR_MISALIGNED;
+    return launch_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, Lq, Lk, d, scale, causal, window_left, window_right,
+                      workspace, workspace_bytes, q_tiles_visited, stream);
+}
+
+int attn_bwd_count_blocks(int Lq, int Lk, int causal, int window_left, int window_right, int block_q, int block_k,
+                          long long* visited) {
+    if (Lq < 1 || Lk < 1 || block_q < 1 || block_k < 1 || !visited) return FATTN_ERR_INVALID_ARG;
+    const Band band = make_band(Lq, Lk, causal, window_left, window_right);
+    *visited = bwd_visited_tiles(band, Lk, block_q, block_k);
     return FATTN_OK;
 }
 

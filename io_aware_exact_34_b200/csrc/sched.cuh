@@ -41,6 +41,12 @@ FATTN_HD Band make_band(long long Lq, long long Lk, int causal, int window_left,
     return b;
 }
 
+// A relative index clamped into [-2^30, 2^30]: far enough outside any tile to
+// compare correctly against tile columns, and safe to offset by a tile width.
+FATTN_HD int clamp_int(long long x) {
+    return (int)(x < -(1LL << 30) ? -(1LL << 30) : (x > (1LL << 30) ? (1LL << 30) : x));
+}
+
 // Visited KV tiles [*lo, *hi) (tiles of bk keys) for the valid query rows
 // [q_first, q_last] of a Q tile.  Empty range: *lo == *hi.
 FATTN_HD void kv_tile_range(const Band& b, long long q_first, long long q_last, int bk,
@@ -61,6 +67,32 @@ FATTN_HD void kv_tile_range(const Band& b, long long q_first, long long q_last, 
     }
     *lo = (int)(jmin / bk);
     *hi = (int)(jmax / bk) + 1;
+}
+
+// The transposed range, for the backward pass that walks Q tiles per KV tile:
+// Q tiles [*lo, *hi) (tiles of bq rows) that hold an allowed pair with the
+// keys [k_first, k_last] (k_last <= Lk - 1).  Key k is allowed for query i
+// iff k - shift - right <= i <= k - shift + left (each side only when
+// bounded), so the queries of the key tile form the interval
+// [k_first - shift - right, k_last - shift + left] clipped to [0, Lq - 1], and
+// every query in it has an allowed key in the tile.  Empty: *lo == *hi.
+FATTN_HD void q_tile_range(const Band& b, long long k_first, long long k_last, int bq, int* lo, int* hi) {
+    long long imin = 0, imax = b.Lq - 1;
+    if (b.right >= 0) {
+        long long t = k_first - b.shift - b.right;
+        imin = t > imin ? t : imin;
+    }
+    if (b.left >= 0) {
+        long long t = k_last - b.shift + b.left;
+        imax = t < imax ? t : imax;
+    }
+    if (k_last < k_first || imax < imin) {
+        *lo = 0;
+        *hi = 0;
+        return;
+    }
+    *lo = (int)(imin / bq);
+    *hi = (int)(imax / bq) + 1;
 }
 
 // True when every (query, key) pair of rows [q_first, q_last] x keys

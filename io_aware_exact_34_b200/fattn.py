@@ -44,6 +44,15 @@ lib.attn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
 lib.attn_decode_workspace_bytes.restype = _sz
 lib.attn_count_blocks.argtypes = [_i, _i, _i, _i, _i, _i, _i, _llp, _llp, _llp, _llp]
 lib.attn_count_blocks.restype = _i
+lib.attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp, _sz, _vp]
+lib.attn_bwd.restype = _i
+lib.attn_bwd_counted.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp,
+                                 _sz, _vp, _vp]
+lib.attn_bwd_counted.restype = _i
+lib.attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i]
+lib.attn_bwd_workspace_bytes.restype = _sz
+lib.attn_bwd_count_blocks.argtypes = [_i, _i, _i, _i, _i, _i, _i, _llp]
+lib.attn_bwd_count_blocks.restype = _i
 lib.fattn_status_string.argtypes = [_i]
 lib.fattn_status_string.restype = ctypes.c_char_p
 lib.fattn_device_status.argtypes = [_vp]
@@ -250,6 +259,47 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seqlens_k, o=None, lse=N
                                  num_pages, _ptr(o), _ptr(lse), _ptr(seqlens_k), B, H, d, scale, S, _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream()), "attn_decode_paged")
     return o, lse
+
+
+def attn_bwd_workspace_bytes(B, H, Lq, d) -> int:
+    return lib.attn_bwd_workspace_bytes(B, H, Lq, d)
+
+
+def attn_bwd(q, k, v, o, dout, lse, scale=None, causal=False, window_left=-1, window_right=-1, dq=None, dk=None,
+             dv=None, workspace=None, counter=None):
+    """Attention backward with recomputation.  q, o, dout: [B,H,Lq,d], k, v:
+    [B,H,Lk,d] bf16; lse: fp32 [B,H,Lq] from attn_fwd -> (dq, dk, dv) bf16.
+    ``counter`` (optional, a zeroed one-element int64 CUDA tensor) receives the
+    number of (key tile, query tile) pairs computed."""
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _want(t, torch.bfloat16, 4, name)
+    _want(lse, torch.float32, 3, "lse")
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if o.shape != q.shape or dout.shape != q.shape or v.shape != k.shape or tuple(lse.shape) != (B, H, Lq):
+        raise ValueError("attn_bwd: inconsistent shapes")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(attn_bwd_workspace_bytes(B, H, Lq, d), dtype=torch.uint8, device=q.device)
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, H, Lq, Lk, d,
+            scale, int(bool(causal)), int(window_left), int(window_right), _ptr(workspace),
+            workspace.numel() * workspace.element_size())
+    if counter is None:
+        _check(lib.attn_bwd(*args, _stream()), "attn_bwd")
+    else:
+        _check(lib.attn_bwd_counted(*args, _ptr(counter), _stream()), "attn_bwd_counted")
+    return dq, dk, dv
+
+
+def attn_bwd_count_blocks(Lq, Lk, causal=False, window_left=-1, window_right=-1, block_q=128, block_k=128) -> int:
+    """Host-side: (query tile, key tile) pairs the backward visits per head."""
+    out = ctypes.c_longlong(0)
+    _check(lib.attn_bwd_count_blocks(Lq, Lk, int(bool(causal)), window_left, window_right, block_q, block_k,
+                                     ctypes.byref(out)), "attn_bwd_count_blocks")
+    return out.value
 
 
 def attn_count_blocks(Lq, Lk, causal=False, window_left=-1, window_right=-1, block_q=128, block_k=128):

@@ -118,6 +118,15 @@ def random_qkv(B, H, Lq, Lk, d, dtype="bf16", seed=0, device="cpu"):
     return make_inputs(w, device=device)
 
 
+def random_dout(B, H, Lq, d, dtype="bf16", seed=0, device="cpu"):
+    """Upstream gradient dO for the backward: i.i.d. N(0, 1), [B, H, Lq, d],
+    from its own generator (seed offset so it never equals a Q draw)."""
+    dev = torch.device(device)
+    g = torch.Generator(device=dev.type)
+    g.manual_seed(1_000_003 + seed)
+    return _draw((B, H, Lq, d), g, dev, _torch_dtype(dtype))
+
+
 def varlen_lengths(n_seqs: int, lo: int, hi: int, seed: int):
     """Sequence lengths drawn uniformly from [lo, hi] (a length mix for packed
     batches of requests)."""

@@ -178,3 +178,46 @@ def test_paged_decode_argument_checks(fl):
     assert call(d=96) == fl.FATTN_ERR_UNSUPPORTED
     assert call(table=FAKE + 2) == fl.FATTN_ERR_MISALIGNED
     assert call(ws=None) == fl.FATTN_ERR_WORKSPACE
+
+
+def _bwd(fl, q=FAKE, k=FAKE, v=FAKE, o=FAKE, do=FAKE, lse=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, B=1, H=2, Lq=300, Lk=260,
+         d=128, scale=0.1, ws=FAKE, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = fl.attn_bwd_workspace_bytes(B, H, Lq, d) if B > 0 and Lq > 0 else 0
+    return fl.lib.attn_bwd(q, k, v, o, do, lse, dq, dk, dv, B, H, Lq, Lk, d, scale, 1, -1, -1, ws, ws_bytes, None)
+
+
+def test_bwd_argument_checks(fl):
+    need = fl.attn_bwd_workspace_bytes(1, 2, 300, 128)
+    assert need == 1 * 2 * 384 * 130 * 4
+    assert fl.attn_bwd_workspace_bytes(1, 1, 1, 96) == 0
+    assert _bwd(fl, lse=None) == fl.FATTN_ERR_INVALID_ARG
+    assert _bwd(fl, do=None) == fl.FATTN_ERR_INVALID_ARG
+    assert _bwd(fl, dq=None) == fl.FATTN_ERR_INVALID_ARG
+    assert _bwd(fl, dk=None) == fl.FATTN_ERR_INVALID_ARG
+    assert _bwd(fl, o=None) == fl.FATTN_ERR_INVALID_ARG
+    assert _bwd(fl, B=0) == fl.FATTN_ERR_INVALID_ARG
+    assert _bwd(fl, scale=0.0) == fl.FATTN_ERR_INVALID_ARG
+    assert _bwd(fl, d=96, ws_bytes=1 << 30) == fl.FATTN_ERR_UNSUPPORTED
+    assert _bwd(fl, do=FAKE + 8) == fl.FATTN_ERR_MISALIGNED
+    assert _bwd(fl, dv=FAKE + 2) == fl.FATTN_ERR_MISALIGNED
+    assert _bwd(fl, lse=FAKE + 2) == fl.FATTN_ERR_MISALIGNED
+    assert _bwd(fl, ws=None) == fl.FATTN_ERR_WORKSPACE
+    assert _bwd(fl, ws_bytes=need - 1) == fl.FATTN_ERR_WORKSPACE
+    assert _bwd(fl, ws=FAKE + 4) == fl.FATTN_ERR_MISALIGNED
+    r = fl.lib.attn_bwd_counted(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 300, 260, 128, 0.1, 1, -1,
+                                -1, FAKE, need, None, None)
+    assert r == fl.FATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
+def test_bwd_valid_call_without_gpu_reports_no_device(fl):
+    assert _bwd(fl) == fl.FATTN_ERR_NO_DEVICE
+
+
+@pytest.mark.parametrize("Lq,Lk,causal,wl,wr,bq,bk", SCHED_CASES)
+def test_bwd_scheduler_matches_bruteforce(fl, oracle, Lq, Lk, causal, wl, wr, bq, bk):
+    """Walking the query tiles of each key tile (the backward's order) visits
+    exactly the tiles with an allowed pair: the oracle's brute-force count."""
+    got = fl.attn_bwd_count_blocks(Lq, Lk, causal, wl, wr, bq, bk)
+    assert got == oracle.count_blocks(Lq, Lk, causal, wl, wr, bq, bk)["visited"]
