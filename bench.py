@@ -53,6 +53,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     "attn_fwd_sm100_kernel": ["attn_fwd_sm100.cuh", "sched.cuh", "dev_prims.cuh"],
     "decode_split_kernel": ["decode_splitkv.cuh", "dev_prims.cuh"],
+    "attn_bwd_sm100_kernel": ["attn_bwd_sm100.cuh", "sched.cuh", "dev_prims.cuh"],
 }
 
 
@@ -349,7 +350,8 @@ def run_ours(args, world, rank, local):
         bwd = {"metric": "attention bwd TFLOP/s (in-mask FLOPs: 10 d per allowed pair)", "value": world * tf,
                "unit": "TFLOP/s", "ms_per_step": bms, "steps": bsteps,
                "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                            "frac": tf / peaks["bf16_tflops"], "traffic": None,
+                            "frac": tf / peaks["bf16_tflops"],
+                            "traffic": recorded_traffic("attn_bwd_sm100_kernel", w.name),
                             "peak_source": f"{peak_src} bf16 dense (burst)",
                             "kernels": ["bwd_prep_kernel", "attn_bwd_sm100_kernel", "bwd_dq_kernel"]},
                "config": {**w.describe(), "pass": "backward with recomputation from LSE"},
