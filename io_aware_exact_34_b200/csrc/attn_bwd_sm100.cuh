@@ -32,7 +32,10 @@
 //   warp 1       MMA issuer (one thread)
 //   warps 4-11   two warpgroups, thread = key row; warpgroup h owns the query
 //                columns [64h, 64h+64) of every score tile: P, dS
-//   warps 12-15  dQ drain, thread = query row: dQ tile -> fp32 atomic adds
+//   warps 12-15  dQ drain, thread = query row: the dQ tile goes from tensor
+//                memory into the stage buffer its Q and dO tiles have left
+//                (the fp32 128 x D tile is exactly their size), then TMA
+//                reduce-adds it into the fp32 accumulator in whole lines
 //
 // Tensor memory (512 columns), lane = key row unless noted:
 //   [0,128)        S^T = K_j Q_i^T (fp32), then P^T (bf16 pairs) over it
@@ -52,6 +55,30 @@
 
 namespace fattn {
 
+// Bytes of per-head working set (Q and dO in bf16, the fp32 dQ accumulator)
+// that the CTAs running at one time should share: heads are scheduled in
+// groups that fit it, so their re-read tiles and accumulator lines stay in L2.
+#ifndef FATTN_BWD_GROUP_BYTES
+#define FATTN_BWD_GROUP_BYTES (16ull << 20)
+#endif
+
+// TMA reduce-add of a 2-D fp32 box from this CTA's shared memory into global
+// memory (whole-line reductions at L2), tracked in the issuing thread's bulk group.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Until every committed bulk operation of this thread has read its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Until every committed bulk operation of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 template <int D>
 struct BwdTraits {
     static constexpr int BQ = 128;                 // queries per Q tile
@@ -68,7 +95,7 @@ struct BwdTraits {
     static constexpr int SMEM_VEC_OFF = SMEM_DS_OFF + DS_BYTES;  // stage s: LSE2 at +0, D at +512
     static constexpr int VEC_STAGE_BYTES = 1024;
     static constexpr int SMEM_BAR_OFF = SMEM_VEC_OFF + NSTAGE * VEC_STAGE_BYTES;
-    static constexpr int NBAR = 1 + 2 * NSTAGE + 8;
+    static constexpr int NBAR = 1 + 2 * NSTAGE + 9;
     static constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NBAR * 8;
     static constexpr int SMEM_USED = SMEM_MISC_OFF + 16;
     // Alignment slack for the 1024-byte aligned base; the kernel checks at run
@@ -79,6 +106,8 @@ struct BwdTraits {
     static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(SMEM_USED <= 232448, "shared memory");
+    // the dQ tile (128 x D fp32) is staged in a stage buffer (Q + dO, 128 x D bf16 each)
+    static_assert(128 * D * 4 == 2 * TILE_BYTES, "dQ staging");
 };
 
 struct BwdParams {
@@ -92,6 +121,7 @@ struct BwdParams {
     float scale, scale_log2;
     int causal, window_left, window_right;
     int reverse;         // 1: launch order takes the last KV tile first
+    int group;           // heads per scheduling group
 };
 
 // ---------------------------------------------------------------- prep
@@ -163,8 +193,9 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ d
 
 // ---------------------------------------------------------------- main kernel
 // Which (bh, KV tile) this CTA owns.  KV tile j runs over the Q tiles
-// [q_lo, q_hi) of the band; the launch takes KV tiles in the order that puts
-// the longest Q ranges first (reverse = 1 walks j downwards).
+// [q_lo, q_hi) of the band.  Heads go in groups of p.group; inside a group the
+// launch takes KV tiles in the order that puts the longest Q ranges first
+// (reverse = 1 walks j downwards), all heads of the group for each j.
 struct BwdTile {
     int bh, j, q_lo, q_hi;
     long long k0, k_last;
@@ -172,8 +203,12 @@ struct BwdTile {
 
 __device__ __forceinline__ BwdTile bwd_tile(const BwdParams& p, const Band& band) {
     BwdTile t;
-    const int jj = blockIdx.x / p.BH;
-    t.bh = blockIdx.x % p.BH;
+    const int per_group = p.group * p.n_kv;
+    const int g = blockIdx.x / per_group;
+    const int r = blockIdx.x - g * per_group;
+    const int gsize = p.BH - g * p.group < p.group ? p.BH - g * p.group : p.group;
+    const int jj = r / gsize;
+    t.bh = g * p.group + (r - jj * gsize);
     t.j = p.reverse ? p.n_kv - 1 - jj : jj;
     t.k0 = static_cast<long long>(t.j) * 128;
     t.k_last = t.k0 + 127 < p.Lk - 1 ? t.k0 + 127 : p.Lk - 1;
@@ -185,7 +220,7 @@ template <int D>
 __global__ void __launch_bounds__(512, 1)
     attn_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                          const BwdParams p) {
+                          const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
     using T = BwdTraits<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -218,6 +253,7 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t dq_empty = dq_full + 8;
     const uint32_t dkdv_full = dq_empty + 8;
     const uint32_t drain_bar = dkdv_full + 8;
+    const uint32_t dq_staged = drain_bar + 8;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + T::SMEM_MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + T::SMEM_MISC_OFF + 4);
 
@@ -229,7 +265,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(kv_full, 1);
         for (int s = 0; s < T::NSTAGE; ++s) {
             mbar_init(qd_full0 + 8 * s, 1);
-            mbar_init(qd_empty0 + 8 * s, 1);
+            mbar_init(qd_empty0 + 8 * s, 2);  // the MMA warp's commit and the dQ drain's release
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
@@ -239,6 +275,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(dq_empty, 128);
         mbar_init(dkdv_full, 1);
         mbar_init(drain_bar, 1);
+        mbar_init(dq_staged, 128);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -247,6 +284,7 @@ __global__ void __launch_bounds__(512, 1)
         tma_prefetch_map(&tm_k);
         tma_prefetch_map(&tm_v);
         tma_prefetch_map(&tm_do);
+        tma_prefetch_map(&tm_dq);
     }
     if (warp == 1) {
         tmem_alloc(smem_addr(tmem_holder), T::TMEM_COLS);
@@ -535,40 +573,53 @@ __global__ void __launch_bounds__(512, 1)
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;  // query row of the dQ tile
         const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + T::TM_DP;
+        const bool leader = warp == 12 && lane == 0;
         bool ok = true;
         for (int n = 0; n < n_tiles && ok; ++n) {
-            const long long i = static_cast<long long>(tile.q_lo + n) * 128 + row;
-            float* acc = p.dq_acc + (static_cast<long long>(tile.bh) * p.Lq_pad + i) * D;
+            const int s = n & 1;
             ok = mbar_wait(dq_full, n & 1u, abort_flag, status, -6);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after_sync();
-            // all of this tile's columns are read before the region is released
-            uint32_t r0[32], r1[32];
+            // dQ(n) has completed, so every MMA that read this stage's Q and dO
+            // tiles has too: the stage buffer takes the fp32 tile, 32 columns
+            // (16 KB, 128-byte rows, 128-byte swizzle) per TMA box
+            uint8_t* stage = gbase + T::SMEM_STAGE_OFF + s * 2 * T::TILE_BYTES;
 #pragma unroll 1
-            for (int ch = 0; ch < D / 32; ch += 2) {
-                tmem_ld32(taddr + ch * 32, r0);
-                tmem_ld32(taddr + ch * 32 + 32, r1);
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t r[32];
+                tmem_ld32(taddr + ch * 32, r);
                 tmem_wait_ld();
-                reg_fence(r0);
-                reg_fence(r1);
-                if (ch + 2 >= D / 32) {
+                reg_fence(r);
+                if (ch == D / 32 - 1) {
+                    // the whole tile is in registers or shared memory: release tensor memory
                     tc_fence_before_sync();
                     mbar_arrive(dq_empty);
                 }
-                if (i < p.Lq) {
+                uint8_t* dst = stage + ch * 16384 + row * 128;
 #pragma unroll
-                    for (int v = 0; v < 8; ++v)
-                        red_add_v4(acc + ch * 32 + 4 * v, __uint_as_float(r0[4 * v]), __uint_as_float(r0[4 * v + 1]),
-                                   __uint_as_float(r0[4 * v + 2]), __uint_as_float(r0[4 * v + 3]));
-#pragma unroll
-                    for (int v = 0; v < 8; ++v)
-                        red_add_v4(acc + ch * 32 + 32 + 4 * v, __uint_as_float(r1[4 * v]),
-                                   __uint_as_float(r1[4 * v + 1]), __uint_as_float(r1[4 * v + 2]),
-                                   __uint_as_float(r1[4 * v + 3]));
+                for (int u = 0; u < 8; ++u)
+                    *reinterpret_cast<uint4*>(dst + ((u ^ (row & 7)) << 4)) =
+                        make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(dq_staged);
+            if (leader) {
+                ok = mbar_wait(dq_staged, n & 1u, abort_flag, status, -6);
+                if (ok) {
+                    const int y = tile.bh * p.Lq_pad + (tile.q_lo + n) * 128;
+                    for (int ch = 0; ch < D / 32; ++ch)
+                        tma_reduce_add_2d(&tm_dq, smem_addr(stage) + ch * 16384, ch * 32, y);
+                    bulk_commit_group();
+                    bulk_wait_read_all();
+                    mbar_arrive(qd_empty0 + 8 * s);  // the stage buffer may be refilled
                 }
             }
+            __syncwarp();
+            ok = __all_sync(0xffffffffu, ok);
         }
+        // the reduce-adds land in the accumulator before the CTA exits
+        if (leader) bulk_wait_all();
     }
 
     // ---------------------------------------------------------------- teardown

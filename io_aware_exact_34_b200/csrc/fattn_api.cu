@@ -154,6 +154,19 @@ int encode_map_packed(CUtensorMap* map, const void* base, int d, int H, long lon
     return r == CUDA_SUCCESS ? FATTN_OK : FATTN_ERR_CUDA;
 }
 
+// The fp32 dQ accumulator as a 2-D [rows, d] tensor: 32-float x 128-row boxes
+// (128-byte rows, 128-byte swizzle) for the backward's TMA reduce-adds.
+int encode_map_acc(CUtensorMap* map, float* base, int d, long long rows) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 4};
+    cuuint32_t box[2] = {32, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FATTN_OK : FATTN_ERR_CUDA;
+}
+
 template <bool kVarlen>
 int launch_prefill_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
                           int d, int grid, cudaStream_t s) {
@@ -285,6 +298,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     float* lse2 = static_cast<float*>(workspace);
     float* dsum = lse2 + BH * Lq_pad;
     float* dq_acc = dsum + BH * Lq_pad;
+    CUtensorMap mdq;
+    if (encode_map_acc(&mdq, dq_acc, d, BH * Lq_pad) != FATTN_OK) return FATTN_ERR_CUDA;
     const Band band = make_band(Lq, Lk, causal, wl, wr);
     BwdParams p;
     p.lse2 = lse2;
@@ -311,6 +326,11 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
         q_tile_range(band, last0, Lk - 1, 128, &lo1, &hi1);
         p.reverse = (hi1 - lo1) > (hi0 - lo0) ? 1 : 0;
     }
+    {
+        const unsigned long long per_head = static_cast<unsigned long long>(Lq_pad) * d * (2 + 2 + 4);
+        const unsigned long long g = FATTN_BWD_GROUP_BYTES / (per_head > 0 ? per_head : 1);
+        p.group = static_cast<int>(g < 1 ? 1 : (g > static_cast<unsigned long long>(BH) ? BH : g));
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const auto* ob = static_cast<const __nv_bfloat16*>(o);
     const auto* dob = static_cast<const __nv_bfloat16*>(dout);
@@ -323,11 +343,11 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     const unsigned grid = static_cast<unsigned>(BH * n_kv);
     if (d == 128) {
         bwd_prep_kernel<128><<<prep_grid, 256, 0, s>>>(ob, dob, lse, lse2, dsum, dq_acc, p.BH, Lq, p.Lq_pad);
-        attn_bwd_sm100_kernel<128><<<grid, BwdTraits<128>::THREADS, BwdTraits<128>::SMEM_BYTES, s>>>(mq, mk, mv, mdo, p);
+        attn_bwd_sm100_kernel<128><<<grid, BwdTraits<128>::THREADS, BwdTraits<128>::SMEM_BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
         bwd_dq_kernel<128><<<fin_grid, 256, 0, s>>>(dq_acc, dqb, p.BH, Lq, p.Lq_pad, scale);
     } else {
         bwd_prep_kernel<64><<<prep_grid, 256, 0, s>>>(ob, dob, lse, lse2, dsum, dq_acc, p.BH, Lq, p.Lq_pad);
-        attn_bwd_sm100_kernel<64><<<grid, BwdTraits<64>::THREADS, BwdTraits<64>::SMEM_BYTES, s>>>(mq, mk, mv, mdo, p);
+        attn_bwd_sm100_kernel<64><<<grid, BwdTraits<64>::THREADS, BwdTraits<64>::SMEM_BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
         bwd_dq_kernel<64><<<fin_grid, 256, 0, s>>>(dq_acc, dqb, p.BH, Lq, p.Lq_pad, scale);
     }
     return cudaGetLastError() == cudaSuccess ? FATTN_OK : FATTN_ERR_CUDA;

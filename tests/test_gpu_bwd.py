@@ -84,6 +84,7 @@ BWD_CASES = [
     (1, 1, 1, 1, 128, False, -1, -1),           # one query, one key
     (2, 1, 7, 7, 64, True, -1, -1),
     (1, 1, 1000, 1, 128, True, -1, -1),         # a single key
+    (1, 4, 5000, 5000, 128, True, -1, -1),      # heads scheduled in groups of 3: a partial last group
 ]
 
 
