@@ -25,6 +25,12 @@
  *       lse = logsumexp_s(lse_s),  o = sum_s exp(lse_s - lse) * o_s.
  *   R7  the tiled recurrence uses m_safe = 0 while the running max is -inf,
  *       otherwise a fully masked first block gives (-inf) - (-inf) = NaN.
+ *   R13 the FP8 forward ("FlashAttention 深度解析" §4 names FlashAttention-3's
+ *       FP8 path and gives no algorithm): Q, K, V are e4m3 codes with one fp32
+ *       descale per (batch, head); scores are the dequantized products; each
+ *       key tile's probabilities, taken against the running row max and
+ *       multiplied by 2^8, are rounded to e4m3 before they weight V; the
+ *       denominator sums the unrounded values.
  *
  * Element types of the inputs: 0 = float64, 1 = float32, 2 = bfloat16 (raw
  * 16-bit patterns).  Every input is widened exactly to double before use, so
@@ -108,9 +114,139 @@ void attend_row(const double* qi, const double* Kd, const double* Vd, long long 
     *lse_out = M + std::log(Z);
 }
 
+/*
+ * The e4m3 format ("fn" variant: no infinities): sign bit, 4 exponent bits
+ * with bias 7, 3 mantissa bits.  Exponent field 0 holds subnormals m * 2^-9;
+ * exponent 15 with mantissa 7 is NaN; the largest finite value is
+ * 1.75 * 2^8 = 448.
+ */
+double e4m3_value(uint8_t code) {
+    const int e = (code >> 3) & 0xF, m = code & 7;
+    if (e == 15 && m == 7) return std::numeric_limits<double>::quiet_NaN();
+    const double mag = e == 0 ? std::ldexp(static_cast<double>(m), -9) : std::ldexp(1.0 + m / 8.0, e - 7);
+    return (code & 0x80) ? -mag : mag;
+}
+
+/* Round to the nearest e4m3 value, ties to the even code, magnitudes above
+ * 448 clamped to 448 (saturating conversion); NaN gives 0x7F.  Plain search
+ * over the 127 finite non-negative codes. */
+uint8_t e4m3_round(double x) {
+    if (std::isnan(x)) return 0x7F;
+    const double a = std::fabs(x);
+    int best = 0;
+    double best_d = std::numeric_limits<double>::infinity();
+    for (int c = 0; c <= 0x7E; ++c) {
+        const double d = std::fabs(e4m3_value(static_cast<uint8_t>(c)) - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    if (a > 448.0) best = 0x7E;
+    return static_cast<uint8_t>(best | (std::signbit(x) ? 0x80 : 0));
+}
+
 }  // namespace
 
 extern "C" {
+
+/* e4m3 codec (pinned against a library conversion in the tests). */
+void oracle_e4m3_decode(const uint8_t* codes, long long n, double* out) {
+    for (long long t = 0; t < n; ++t) out[t] = e4m3_value(codes[t]);
+}
+
+void oracle_e4m3_encode(const double* x, long long n, uint8_t* out) {
+    for (long long t = 0; t < n; ++t) out[t] = e4m3_round(x[t]);
+}
+
+/*
+ * Per-group FP8 quantization: for each of `groups` runs of `group_len`
+ * elements, amax = max |x|, descale = amax / 448 and code = e4m3(x * (448 /
+ * amax)), where the reciprocal scale and the product are each one fp32
+ * operation rounded to nearest (the precision the kernel decides in); a group
+ * of zeros gets descale 1.  x is widened from its stored type to fp32 first.
+ */
+void oracle_quantize_fp8(const void* x, int dtype, long long groups, long long group_len, uint8_t* codes,
+                         float* descale) {
+    for (long long g = 0; g < groups; ++g) {
+        float amax = 0.0f;
+        for (long long t = 0; t < group_len; ++t)
+            amax = std::max(amax, std::fabs(static_cast<float>(widen(x, g * group_len + t, dtype))));
+        const volatile float four48 = 448.0f;
+        const float inv = amax > 0.0f ? four48 / amax : 1.0f;
+        descale[g] = amax > 0.0f ? amax / four48 : 1.0f;
+        for (long long t = 0; t < group_len; ++t) {
+            const volatile float y = static_cast<float>(widen(x, g * group_len + t, dtype)) * inv;
+            codes[g * group_len + t] = e4m3_round(static_cast<double>(y));
+        }
+    }
+}
+
+/*
+ * FP8 forward by the steps of reading R13 on the tiled online softmax of
+ * [P2] §3.2, one query row at a time over key tiles of block_k keys:
+ *   x_j   = scale * qd * kd * (q8_i . k8_j) * log2(e)      (allowed keys)
+ *   m'    = max(m, max_j x_j);  alpha = 2^(m - m');  l, acc *= alpha
+ *   p_j   = 2^(x_j - m' + 8);   l += p_j
+ *   acc  += e4m3(p_j) * v8_j    (p_j itself when quantize_p == 0)
+ * and at the end O = vd * acc / l, LSE = ln2 * (m + log2 l - 8).  q8, k8, v8
+ * are e4m3 codes [B,H,L,d]; qd, kd, vd the per-(b,h) descales.  A row with no
+ * allowed key gets O = 0 and LSE = -inf.
+ */
+void oracle_attn_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* qd, const float* kd,
+                     const float* vd, double* o, double* lse, int B, int H, int Lq, int Lk, int d, double scale,
+                     int causal, int wl, int wr, int block_k, int quantize_p) {
+    const double LOG2E = 1.4426950408889634074;
+    for (long long bh = 0; bh < static_cast<long long>(B) * H; ++bh) {
+        std::vector<double> Kd(static_cast<size_t>(Lk) * d), Vd(static_cast<size_t>(Lk) * d);
+        for (long long t = 0; t < static_cast<long long>(Lk) * d; ++t) {
+            Kd[t] = e4m3_value(k8[bh * Lk * d + t]);
+            Vd[t] = e4m3_value(v8[bh * Lk * d + t]);
+        }
+        const double c = scale * static_cast<double>(qd[bh]) * static_cast<double>(kd[bh]) * LOG2E;
+#pragma omp parallel for schedule(dynamic, 16)
+        for (int i = 0; i < Lq; ++i) {
+            std::vector<double> qi(d), acc(d, 0.0), x(block_k);
+            std::vector<char> ok(block_k);
+            for (int e = 0; e < d; ++e) qi[e] = e4m3_value(q8[(bh * Lq + i) * d + e]);
+            double m = NEG_INF, l = 0.0;
+            for (long long k0 = 0; k0 < Lk; k0 += block_k) {
+                const int n = static_cast<int>(std::min<long long>(block_k, Lk - k0));
+                double mx = NEG_INF;
+                for (int t = 0; t < n; ++t) {
+                    ok[t] = allowed(i, k0 + t, Lq, Lk, Lk, causal, wl, wr);
+                    if (!ok[t]) continue;
+                    double dot = 0.0;
+                    for (int e = 0; e < d; ++e) dot += qi[e] * Kd[(k0 + t) * d + e];
+                    x[t] = c * dot;
+                    mx = std::max(mx, x[t]);
+                }
+                if (mx == NEG_INF) continue;  /* no allowed key of this row in the tile */
+                if (mx > m) {
+                    const double alpha = m == NEG_INF ? 0.0 : std::exp2(m - mx);
+                    l *= alpha;
+                    for (int e = 0; e < d; ++e) acc[e] *= alpha;
+                    m = mx;
+                }
+                for (int t = 0; t < n; ++t) {
+                    if (!ok[t]) continue;
+                    const double p = std::exp2(x[t] - m + 8.0);
+                    l += p;
+                    const double pq = quantize_p ? e4m3_value(e4m3_round(p)) : p;
+                    for (int e = 0; e < d; ++e) acc[e] += pq * Vd[(k0 + t) * d + e];
+                }
+            }
+            const long long row = bh * Lq + i;
+            if (l == 0.0) {
+                for (int e = 0; e < d; ++e) o[row * d + e] = 0.0;
+                lse[row] = NEG_INF;
+                continue;
+            }
+            for (int e = 0; e < d; ++e) o[row * d + e] = static_cast<double>(vd[bh]) * acc[e] / l;
+            lse[row] = std::log(2.0) * (m + std::log2(l) - 8.0);
+        }
+    }
+}
 
 int oracle_num_threads(void) { return omp_get_max_threads(); }
 

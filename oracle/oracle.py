@@ -52,6 +52,13 @@ def _load():
             lib.oracle_decode_splitmerge.argtypes = [vp, vp, vp, i, dp, dp, i, i, i, i, d, ip, i]
             lib.oracle_count_blocks.argtypes = [i, i, i, i, i, i, i, llp, llp, llp, llp]
             lib.oracle_attn_bwd.argtypes = [vp, vp, vp, vp, i, dp, dp, dp, i, i, i, i, i, d, i, i, i]
+            u8p = ctypes.POINTER(ctypes.c_uint8)
+            fp = ctypes.POINTER(ctypes.c_float)
+            ll = ctypes.c_longlong
+            lib.oracle_e4m3_decode.argtypes = [u8p, ll, dp]
+            lib.oracle_e4m3_encode.argtypes = [dp, ll, u8p]
+            lib.oracle_quantize_fp8.argtypes = [vp, i, ll, ll, u8p, fp]
+            lib.oracle_attn_fp8.argtypes = [u8p, u8p, u8p, fp, fp, fp, dp, dp, i, i, i, i, i, d, i, i, i, i, i]
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_set_num_threads.argtypes = [i]
             _lib = lib
@@ -210,6 +217,60 @@ def attn_bwd(q, k, v, do, scale, causal=False, window_left=-1, window_right=-1):
                             B, H, Lq, Lk, d, float(scale), int(bool(causal)), int(window_left),
                             int(window_right))
     return dq, dk, dv
+
+
+def _u8(a):
+    a = np.ascontiguousarray(a, dtype=np.uint8)
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+
+
+def _f32(a):
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+
+
+def e4m3_decode(codes):
+    """Values (float64) of e4m3 codes (uint8 array)."""
+    c, cp = _u8(codes)
+    out = np.empty(c.shape, np.float64)
+    _load().oracle_e4m3_decode(cp, c.size, _dptr(out))
+    return out
+
+
+def e4m3_encode(x):
+    """Nearest e4m3 codes (ties to even, saturating at 448) of float64 values."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(x.shape, np.uint8)
+    _load().oracle_e4m3_encode(_dptr(x), x.size, out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    return out
+
+
+def quantize_fp8(x):
+    """Per-(b,h) FP8 quantization of x [B,H,L,d] -> (codes uint8 [B,H,L,d],
+    descale float32 [B,H])."""
+    xa, dt = _as_array(x)
+    B, H, L, d = xa.shape
+    codes = np.empty((B, H, L, d), np.uint8)
+    desc = np.empty((B, H), np.float32)
+    _load().oracle_quantize_fp8(_ptr(xa), dt, B * H, L * d, codes.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+                                desc.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    return codes, desc
+
+
+def attn_fp8(q8, k8, v8, qd, kd, vd, scale, causal=False, window_left=-1, window_right=-1, block_k=128,
+             quantize_p=True):
+    """FP8 forward by its steps (e4m3 codes [B,H,L,d], per-(b,h) descales) ->
+    (O [B,H,Lq,d] float64, LSE [B,H,Lq] float64)."""
+    (q8, qp), (k8, kp), (v8, vp) = _u8(q8), _u8(k8), _u8(v8)
+    (qd, qdp), (kd, kdp), (vd, vdp) = _f32(qd), _f32(kd), _f32(vd)
+    B, H, Lq, d = q8.shape
+    Lk = k8.shape[2]
+    o = np.empty((B, H, Lq, d), np.float64)
+    lse = np.empty((B, H, Lq), np.float64)
+    _load().oracle_attn_fp8(qp, kp, vp, qdp, kdp, vdp, _dptr(o), _dptr(lse), B, H, Lq, Lk, d, float(scale),
+                            int(bool(causal)), int(window_left), int(window_right), int(block_k),
+                            int(bool(quantize_p)))
+    return o, lse
 
 
 def count_blocks(Lq, Lk, causal, window_left, window_right, block_q, block_k):
