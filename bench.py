@@ -8,7 +8,7 @@ Q/K/V tiles, tcgen05 S = Q K^T, masked exp2 online softmax, P V, O / l and
 LSE) over the causal 4 x 16 x 4096, d = 128 bf16 workload; ``value`` is its
 in-mask TFLOP/s (4 d FLOPs per allowed (q, k) pair per head) with inputs
 resident in HBM.  The same run times the backward with recomputation on that
-workload (``bwd``), the split-KV decode path (split kernel + LSE merge) on the
+workload (``bwd``), the FP8 forward on it (``fp8``), the split-KV decode path (split kernel + LSE merge) on the
 64 x 32 x 32768 cache under ``decode`` in GB/s of K/V/q/o/lse traffic, and the
 sliding-window / long-causal prefill workloads under ``extra``.
 
@@ -359,6 +359,40 @@ def run_ours(args, world, rank, local):
         del dout, gq, gk, gv, gws
         torch.cuda.empty_cache()
 
+    # ---------------------------------------------------------------- FP8 forward
+    fp8 = None
+    if not args.no_fp8:
+        q8, qs = fattn.attn_quantize_fp8(q)
+        k8, ks = fattn.attn_quantize_fp8(k)
+        vt8, vs = fattn.attn_quantize_fp8(v, transpose=True)
+        o8 = torch.empty_like(o)
+
+        def fstep():
+            fattn.attn_fwd_fp8(q8, k8, vt8, qs, ks, vs, o=o8, lse=lse, scale=w.scale, causal=w.causal,
+                               window_left=w.window_left, window_right=w.window_right)
+
+        def qstep():
+            fattn.attn_quantize_fp8(q, codes=q8, descale=qs)
+            fattn.attn_quantize_fp8(k, codes=k8, descale=ks)
+            fattn.attn_quantize_fp8(v, transpose=True, codes=vt8, descale=vs)
+
+        fsteps = max(3, min(args.steps, 20))
+        fms = timed(world, fstep, fsteps, 3)
+        qms = timed(world, qstep, 3, 3)
+        tf = flops / (fms * 1e-3) / 1e12
+        fp8_peak = 2.0 * peaks["bf16_tflops"]  # nominal dense fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s)
+        fp8 = {"metric": "attention fwd TFLOP/s (in-mask FLOPs), e4m3 Q/K/V/P", "value": world * tf,
+               "unit": "TFLOP/s", "ms_per_step": fms, "steps": fsteps,
+               "roofline": {"bound": "tensor", "achieved": tf, "peak": fp8_peak, "unit": "TFLOP/s",
+                            "frac": tf / fp8_peak, "traffic": None,
+                            "peak_source": f"{peak_src} bf16 dense (burst) x 2 (nominal fp8/bf16 ratio)",
+                            "kernel": PREFILL_KERNEL + "<128, false, true>"},
+               "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
+               "quantize_ms_per_step": qms, "config": {**w.describe(), "dtype": "e4m3 (P e4m3, O bf16)"},
+               "gpu_launches": fsteps}
+        del q8, k8, vt8, qs, ks, vs, o8
+        torch.cuda.empty_cache()
+
     # ---------------------------------------------------------------- decode
     decode = None
     if not args.no_decode:
@@ -475,7 +509,7 @@ def run_ours(args, world, rank, local):
                            "kv_tiles_visited_per_head": counts["visited"],
                            "kv_tiles_total_per_head": counts["total"]},
                 "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
-                "clocks": clocks, "bwd": bwd, "decode": decode, "decode_paged": decode_paged, "extra": extra,
+                "clocks": clocks, "bwd": bwd, "fp8": fp8, "decode": decode, "decode_paged": decode_paged, "extra": extra,
                 "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)
 
@@ -492,6 +526,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -134,6 +134,64 @@ int attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float
                  int causal, int window_left, int window_right, void* stream);
 
 /*
+ * attn_fwd_fp8 -- the prefill forward with 8-bit (e4m3) Q, K and V on the
+ * tensor cores' kind::f8f6f4 path ("FlashAttention 深度解析" §4 names
+ * FlashAttention-3's FP8 path; this is the plain reading of it on the tiled
+ * online softmax): S = Q K^T from the e4m3 codes with fp32 accumulation,
+ * x = S * scale * q_descale * k_descale; against the exact running row max m,
+ * p = 2^(x*log2e - m + 8) is rounded to e4m3 (nearest, ties to even) before
+ * the P V product; l sums the unrounded p; O = v_descale * acc / l (bf16) and
+ * LSE = ln2 (m + log2 l - 8) (fp32, natural log).  Mask as attn_fwd.
+ *
+ *   q8         device, e4m3 codes [B,H,Lq,128]
+ *   k8         device, e4m3 codes [B,H,Lk,128]
+ *   vt8        device, e4m3 codes of V transposed, [B,H,128,ld] with
+ *              ld = attn_fp8_ld(Lk) (Lk rounded up to 16); columns >= Lk ignored
+ *   q_descale, k_descale, v_descale
+ *              device, fp32 [B*H]: the value of code c of head (b,h) is
+ *              e4m3(c) * descale[b*H + h] (attn_quantize_fp8 writes them)
+ *   o, lse     device, bf16 [B,H,Lq,128] / fp32 [B,H,Lq] (lse nullable)
+ *   d          must be 128 (FATTN_ERR_UNSUPPORTED otherwise)
+ * Tensors 16-byte aligned, descales 4-byte aligned.
+ *
+ * Accuracy against exact attention on the dequantized inputs: rounding p to
+ * e4m3 changes each weight by at most 2^-4 of itself (2^-10 absolute below
+ * e4m3's normal range), so a row's O moves by at most about
+ * 2^-4 * max|v| and, for rows spread over many keys, far less.
+ */
+int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8,
+                 const float* q_descale, const float* k_descale, const float* v_descale,
+                 void* o, float* lse, int B, int H, int Lq, int Lk, int d, float scale,
+                 int causal, int window_left, int window_right, void* stream);
+
+/* attn_fwd_fp8 that also counts the KV tiles visited (see attn_fwd_counted). */
+int attn_fwd_fp8_counted(const void* q8, const void* k8, const void* vt8,
+                         const float* q_descale, const float* k_descale, const float* v_descale,
+                         void* o, float* lse, int B, int H, int Lq, int Lk, int d, float scale,
+                         int causal, int window_left, int window_right,
+                         unsigned long long* kv_tiles_visited, void* stream);
+
+/* Row length of attn_fwd_fp8's transposed V: Lk rounded up to a multiple of
+ * 16 (0 for Lk < 1).  Host only. */
+int attn_fp8_ld(int Lk);
+
+/*
+ * attn_quantize_fp8 -- bf16 -> e4m3 with one scale per (batch, head):
+ * amax = max |x| over the head, code = e4m3(x * (448 / amax)) with the
+ * reciprocal and the product each one fp32 operation rounded to nearest
+ * (nearest-even, saturating conversion), descale = amax / 448 (1 for a head
+ * of zeros).
+ *
+ *   x          device, bf16 [B,H,L,d], d in {64, 128}
+ *   codes      device, e4m3 [B,H,L,d] (transpose = 0) or [B,H,d,ld] with
+ *              ld = attn_fp8_ld(L), columns >= L written as 0 (transpose = 1)
+ *   descale    device, fp32 [B*H] (written)
+ * B*H <= 65535.  Four kernels (and a memset of descale) are enqueued.
+ */
+int attn_quantize_fp8(const void* x, void* codes, float* descale, int B, int H, int L, int d,
+                      int transpose, void* stream);
+
+/*
  * attn_decode_splitkv -- split-KV decode for one new query per sequence (flash
  * decoding: "算子与编译器：FlashAttention 与长上下文" §4, short query and long
  * K/V, parallel along the KV axis).  Split s of num_splits covers keys

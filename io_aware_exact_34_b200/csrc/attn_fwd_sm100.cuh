@@ -29,6 +29,16 @@
 // denominator use the same reference, so O = acc / l is unchanged (the page's
 // "skipped block == all -inf block" argument of §5.5 generalises to any
 // common reference), and O in TMEM is rescaled only when the reference moves.
+//
+// FP8 instantiation (kFp8): Q, K are e4m3 [B,H,L,128] and V is e4m3 stored
+// transposed, [B,H,128,ldv], so both products read K-major operands; one fp32
+// descale per (b,h) for each of Q, K, V.  S = Q K^T and O += P V run as
+// kind::f8f6f4 MMAs (32 elements of K per instruction).  The running max is
+// exact (no slack) and p = 2^(x - m + 8) <= 2^8 is rounded to e4m3 before the
+// P V product, so typical probabilities sit in e4m3's normal range; l sums the
+// unrounded p; O = vd * acc / l and LSE = ln2 (m + log2 l - 8).  This is the
+// FP8 path FlashAttention-3 is named for in "FlashAttention 深度解析" §4,
+// taken on the tiled recurrence above.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -41,14 +51,16 @@ namespace fattn {
 
 constexpr float kRescaleSlack = 8.0f;
 
-template <int D>
+template <int D, bool kFp8 = false>
 struct FwdTraits {
+    static constexpr int ELEM = kFp8 ? 1 : 2;      // bytes per element
     static constexpr int BQ = 128;                 // rows per Q tile (one per TMEM lane)
     static constexpr int BK = 128;                 // keys per KV tile
-    static constexpr int CHUNK_BYTES = 128 * 128;  // 128 rows x 64 bf16: one 128-B swizzle column
-    static constexpr int NCHUNK = D / 64;
-    static constexpr int TILE_BYTES = 128 * D * 2;
-    static constexpr int NSTAGE = D == 128 ? 4 : 8;  // K/V ring slots
+    static constexpr int CHUNK_BYTES = 128 * 128;  // 128 rows x 128 B: one 128-B swizzle column
+    static constexpr int NCHUNK = D * ELEM / 128;
+    static constexpr int TILE_BYTES = 128 * D * ELEM;
+    static constexpr int NSTAGE = TILE_BYTES == 32768 ? 4 : 8;  // K/V ring slots
+    static constexpr int KSTEPS_S = D * ELEM / 32;              // 32-byte K steps of S = Q K^T
     static constexpr int SMEM_Q_OFF = 0;
     static constexpr int SMEM_RING_OFF = 2 * TILE_BYTES;
     static constexpr int SMEM_BAR_OFF = SMEM_RING_OFF + NSTAGE * TILE_BYTES;
@@ -69,6 +81,7 @@ struct FwdTraits {
     __host__ __device__ static constexpr uint32_t tm_s(int t) { return static_cast<uint32_t>(t) * 128u; }
     __host__ __device__ static constexpr uint32_t tm_o(int t) { return 256u + static_cast<uint32_t>(t) * D; }
     static_assert(D == 64 || D == 128, "head dim");
+    static_assert(!kFp8 || D == 128, "the FP8 path is built for d = 128");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
@@ -86,6 +99,10 @@ struct FwdParams {
     const int* cu_q;
     const int* cu_k;
     int total_q, total_k;
+    // FP8 path: per-(b,h) descales of Q, K, V
+    const float* q_descale;
+    const float* k_descale;
+    const float* v_descale;
 };
 
 // The sequence and head of one work item: its pair index, token offsets and
@@ -251,6 +268,35 @@ __device__ __forceinline__ float softmax_tile_probs(const uint32_t (&sr)[4][32],
     return lo + hi;
 }
 
+// FP8 variant: p_c = 2^(s_c * c_log2 - m_shift) (m_shift = m_safe - 8, so
+// p_c <= 2^8), rounded to e4m3 four to a word (key 4i in the low byte of
+// pk[i]); returns the fp32 sum of the unrounded p_c.  Masked scores (-inf)
+// give exactly 0.
+__device__ __forceinline__ float softmax_tile_probs_fp8(const uint32_t (&sr)[4][32], uint32_t (&pk)[32], float c_log2,
+                                                        float m_shift) {
+    const uint64_t scale2 = f2_pack(c_log2, c_log2);
+    const uint64_t shift2 = f2_pack(-m_shift, -m_shift);
+    uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int c = 4 * i;
+        const uint64_t x01 = f2_fma(f2_pack(__uint_as_float(sr[c >> 5][c & 31]), __uint_as_float(sr[c >> 5][(c & 31) + 1])),
+                                    scale2, shift2);
+        const uint64_t x23 = f2_fma(f2_pack(__uint_as_float(sr[c >> 5][(c & 31) + 2]), __uint_as_float(sr[c >> 5][(c & 31) + 3])),
+                                    scale2, shift2);
+        float x0, x1, x2, x3;
+        f2_unpack(x01, x0, x1);
+        f2_unpack(x23, x2, x3);
+        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1), p2 = fast_exp2(x2), p3 = fast_exp2(x3);
+        sum2[i & 3] = f2_add(sum2[i & 3], f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
+        pk[i] = pack_e4m3x4(p0, p1, p2, p3);
+    }
+    const uint64_t s01 = f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3]));
+    float lo, hi;
+    f2_unpack(s01, lo, hi);
+    return lo + hi;
+}
+
 // Row max of 128 scores with four independent 3-input max chains.
 __device__ __forceinline__ float row_max128(const uint32_t (&sr)[4][32]) {
     float m[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
@@ -262,11 +308,12 @@ __device__ __forceinline__ float row_max128(const uint32_t (&sr)[4][32]) {
     return fmax3(m[0], m[1], fmaxf(m[2], m[3]));
 }
 
-template <int D, bool kVarlen>
+template <int D, bool kVarlen, bool kFp8 = false>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using T = FwdTraits<D>;
+    using T = FwdTraits<D, kFp8>;
+    static_assert(!(kFp8 && kVarlen), "the FP8 path takes dense batches");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -338,7 +385,7 @@ __global__ void __launch_bounds__(384, 1)
                 mbar_arrive_expect_tx(q_full, 2 * T::TILE_BYTES);
                 for (int t = 0; t < 2; ++t)
                     for (int c = 0; c < T::NCHUNK; ++c)
-                        tma_load_3d(sQ + t * T::TILE_BYTES + c * T::CHUNK_BYTES, &tm_q, q_full, c * 64,
+                        tma_load_3d(sQ + t * T::TILE_BYTES + c * T::CHUNK_BYTES, &tm_q, q_full, c * (128 / T::ELEM),
                                     kVarlen ? ts.h : ts.q_first[t], kVarlen ? ts.q_start + ts.q_first[t] : ts.bh);
                 ++q_round;
                 for (int j = ts.lo; j < ts.hi && ok; ++j) {
@@ -356,9 +403,15 @@ __global__ void __launch_bounds__(384, 1)
                         }
                         const uint32_t fb = kv_full0 + 8 * slot;
                         mbar_arrive_expect_tx(fb, T::TILE_BYTES);
-                        for (int c = 0; c < T::NCHUNK; ++c)
-                            tma_load_3d(sRing + slot * T::TILE_BYTES + c * T::CHUNK_BYTES, kv ? &tm_v : &tm_k, fb,
-                                        c * 64, kVarlen ? ts.h : j * 128, kVarlen ? ts.k_start + j * 128 : ts.bh);
+                        if (kFp8 && kv) {
+                            // V^T tile: 128 keys (x, contiguous) of all 128 d rows
+                            tma_load_3d(sRing + slot * T::TILE_BYTES, &tm_v, fb, j * 128, 0, ts.bh);
+                        } else {
+                            for (int c = 0; c < T::NCHUNK; ++c)
+                                tma_load_3d(sRing + slot * T::TILE_BYTES + c * T::CHUNK_BYTES, kv ? &tm_v : &tm_k, fb,
+                                            c * (128 / T::ELEM), kVarlen ? ts.h : j * 128,
+                                            kVarlen ? ts.k_start + j * 128 : ts.bh);
+                        }
                         ++ring;
                     }
                 }
@@ -375,8 +428,9 @@ __global__ void __launch_bounds__(384, 1)
       } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+            constexpr uint32_t idesc_s = kFp8 ? idesc_e4m3_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 128, 0, 0);
+            // FP8: V^T is K-major; bf16: V is MN-major (d contiguous)
+            constexpr uint32_t idesc_pv = kFp8 ? idesc_e4m3_f32(128, D, 0, 0) : idesc_bf16_f32(128, D, 0, 1);
             uint32_t ring = 0, q_round = 0, p_cnt[2] = {0u, 0u};
             bool ok = true;
             for (int round = 0; ok; ++round) {
@@ -405,14 +459,25 @@ __global__ void __launch_bounds__(384, 1)
                             ++p_cnt[t];
                             if (!ok) break;
                             tc_fence_after_sync();
-                            const uint32_t v_lo = sdesc_lo(sRing + (rV % T::NSTAGE) * T::TILE_BYTES, T::CHUNK_BYTES);
                             const uint32_t first = (j - 1 == ts.lo_t[t]) ? 1u : 0u;
+                            if constexpr (kFp8) {
+                                const uint32_t v_lo = sdesc_lo(sRing + (rV % T::NSTAGE) * T::TILE_BYTES, 16);
 #pragma unroll
-                            for (int ks = 0; ks < 8; ++ks) {
-                                // 16 keys = 16 rows of 128 B further into the V tile
-                                mma_bf16_ts(tmem + T::tm_o(t), tmem + T::tm_s(t) + ks * 8,
-                                            sdesc_from_lo(v_lo + ks * (2048 >> 4)), idesc_pv,
-                                            (first && ks == 0) ? 0u : 1u);
+                                for (int ks = 0; ks < 4; ++ks) {
+                                    // 32 keys = 8 TMEM columns of packed P, 32 B along the V^T rows
+                                    mma_fp8_ts(tmem + T::tm_o(t), tmem + T::tm_s(t) + ks * 8,
+                                               sdesc_from_lo(v_lo + ks * (32 >> 4)), idesc_pv,
+                                               (first && ks == 0) ? 0u : 1u);
+                                }
+                            } else {
+                                const uint32_t v_lo = sdesc_lo(sRing + (rV % T::NSTAGE) * T::TILE_BYTES, T::CHUNK_BYTES);
+#pragma unroll
+                                for (int ks = 0; ks < 8; ++ks) {
+                                    // 16 keys = 16 rows of 128 B further into the V tile
+                                    mma_bf16_ts(tmem + T::tm_o(t), tmem + T::tm_s(t) + ks * 8,
+                                                sdesc_from_lo(v_lo + ks * (2048 >> 4)), idesc_pv,
+                                                (first && ks == 0) ? 0u : 1u);
+                                }
                             }
                             if (j - 1 == ts.hi_t[t] - 1) mma_commit(o_full0 + 8 * t);
                         }
@@ -421,11 +486,15 @@ __global__ void __launch_bounds__(384, 1)
                             const uint32_t k_lo = sdesc_lo(sRing + (rK % T::NSTAGE) * T::TILE_BYTES, 16);
                             const uint32_t q_lo = sdesc_lo(sQ + t * T::TILE_BYTES, 16);
 #pragma unroll
-                            for (int ks = 0; ks < D / 16; ++ks) {
-                                // 16 elements = 32 B along the swizzled row; 64 elements = next 16 KB column
+                            for (int ks = 0; ks < T::KSTEPS_S; ++ks) {
+                                // 32 B along the swizzled row per step; every 128 B the next 16 KB column
                                 const uint32_t off = ((ks / 4) * T::CHUNK_BYTES + (ks % 4) * 32) >> 4;
-                                mma_bf16_ss(tmem + T::tm_s(t), sdesc_from_lo(q_lo + off), sdesc_from_lo(k_lo + off),
-                                            idesc_s, ks > 0 ? 1u : 0u);
+                                if constexpr (kFp8)
+                                    mma_fp8_ss(tmem + T::tm_s(t), sdesc_from_lo(q_lo + off), sdesc_from_lo(k_lo + off),
+                                               idesc_s, ks > 0 ? 1u : 0u);
+                                else
+                                    mma_bf16_ss(tmem + T::tm_s(t), sdesc_from_lo(q_lo + off), sdesc_from_lo(k_lo + off),
+                                                idesc_s, ks > 0 ? 1u : 0u);
                             }
                             mma_commit(s_full0 + 8 * t);
                         }
@@ -451,7 +520,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t taddr_s = tmem + lane_off + T::tm_s(t);
         const uint32_t taddr_o = tmem + lane_off + T::tm_o(t);
         const uint32_t s_full = s_full0 + 8 * t, p_ready = p_ready0 + 8 * t, o_full = o_full0 + 8 * t;
-        const float c_log2 = p.scale_log2;
+        constexpr float slack = kFp8 ? 0.0f : kRescaleSlack;
         uint32_t s_phase = 0, o_phase = 0;
         bool ok = true;
         for (int round = 0; ok; ++round) {
@@ -459,6 +528,12 @@ __global__ void __launch_bounds__(384, 1)
             if (item >= p.n_items) break;
             const RowPlan rp = row_plan<D, kVarlen>(p, item, t, row);
             if (!rp.tile_exists) continue;
+            float c_log2 = p.scale_log2, o_scale = 1.f;
+            if constexpr (kFp8) {
+                const int bh = item_seq<kVarlen>(p, item).bh;
+                c_log2 *= __ldg(p.q_descale + bh) * __ldg(p.k_descale + bh);
+                o_scale = __ldg(p.v_descale + bh);
+            }
             if (rp.lo >= rp.hi) {
                 // no allowed key for any row of this tile
                 if (rp.valid) {
@@ -494,22 +569,28 @@ __global__ void __launch_bounds__(384, 1)
                 const float mx_s = row_max128(sr) * c_log2;
                 float alpha = 1.f;
                 bool resc = false;
-                if (mx_s > m_used + kRescaleSlack) {
+                if (mx_s > m_used + slack) {
                     alpha = fast_exp2(m_used - mx_s);  // 0 when m_used is -inf
                     resc = (j > rp.lo) && (m_used != -CUDART_INF_F);
                     m_used = mx_s;
                     l *= alpha;
                 }
                 const float m_safe = (m_used == -CUDART_INF_F) ? 0.f : m_used;
-                uint32_t pk[2][32];
-                float rowsum;
-                if (full_tile)
-                    rowsum = softmax_tile_probs<true>(sr, pk, c_log2, m_safe);
-                else
-                    rowsum = softmax_tile_probs<false>(sr, pk, c_log2, m_safe);
-                l += rowsum;
-                tmem_st32(taddr_s, pk[0]);
-                tmem_st32(taddr_s + 32, pk[1]);
+                if constexpr (kFp8) {
+                    uint32_t pk8[32];
+                    l += softmax_tile_probs_fp8(sr, pk8, c_log2, m_safe - 8.f);
+                    tmem_st32(taddr_s, pk8);
+                } else {
+                    uint32_t pk[2][32];
+                    float rowsum;
+                    if (full_tile)
+                        rowsum = softmax_tile_probs<true>(sr, pk, c_log2, m_safe);
+                    else
+                        rowsum = softmax_tile_probs<false>(sr, pk, c_log2, m_safe);
+                    l += rowsum;
+                    tmem_st32(taddr_s, pk[0]);
+                    tmem_st32(taddr_s + 32, pk[1]);
+                }
                 if (__any_sync(0xffffffffu, resc)) {
                     const float a = resc ? alpha : 1.f;
 #pragma unroll 1
@@ -534,7 +615,7 @@ __global__ void __launch_bounds__(384, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after_sync();
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            const float inv_l = l > 0.f ? o_scale / l : 0.f;
             __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + rp.o_off;
 #pragma unroll 1
             for (int ch = 0; ch < D / 32; ++ch) {
@@ -552,7 +633,8 @@ __global__ void __launch_bounds__(384, 1)
                     for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk16[4 * v], pk16[4 * v + 1], pk16[4 * v + 2], pk16[4 * v + 3]);
                 }
             }
-            if (rp.valid && p.lse) p.lse[rp.lse_off] = l > 0.f ? (m_used + __log2f(l)) * 0.6931471805599453f : -CUDART_INF_F;
+            if (rp.valid && p.lse)
+                p.lse[rp.lse_off] = l > 0.f ? (m_used + __log2f(l) - (kFp8 ? 8.f : 0.f)) * 0.6931471805599453f : -CUDART_INF_F;
             if (p.visited && quarter == 0 && lane == 0)
                 atomicAdd(p.visited, static_cast<unsigned long long>(rp.hi - rp.lo));
         }

@@ -18,6 +18,7 @@
 #include "attn_fwd_f32.cuh"
 #include "attn_fwd_sm100.cuh"
 #include "decode_splitkv.cuh"
+#include "fp8_quant.cuh"
 #include "sched.cuh"
 
 namespace {
@@ -38,15 +39,17 @@ struct DeviceInfo {
 // raising warpgroups would wait forever.  Checked against the compiled kernel.
 template <int D>
 bool fwd_register_pool_ok() {
-    cudaFuncAttributes a, b;
+    cudaFuncAttributes a, b, c;
     if (cudaFuncGetAttributes(&a, attn_fwd_sm100_kernel<D, false>) != cudaSuccess ||
-        cudaFuncGetAttributes(&b, attn_fwd_sm100_kernel<D, true>) != cudaSuccess) {
+        cudaFuncGetAttributes(&b, attn_fwd_sm100_kernel<D, true>) != cudaSuccess ||
+        cudaFuncGetAttributes(&c, attn_fwd_sm100_kernel<128, false, true>) != cudaSuccess) {
         cudaGetLastError();
         return false;
     }
     using T = FwdTraits<D>;
     const long long need = 128LL * T::REGS_LOW + 256LL * T::REGS_HIGH;
-    return static_cast<long long>(a.numRegs) * T::THREADS >= need && static_cast<long long>(b.numRegs) * T::THREADS >= need;
+    return static_cast<long long>(a.numRegs) * T::THREADS >= need && static_cast<long long>(b.numRegs) * T::THREADS >= need &&
+           static_cast<long long>(c.numRegs) * T::THREADS >= need;
 }
 
 std::mutex g_mutex;
@@ -88,6 +91,7 @@ int device_ready(DeviceInfo* out) {
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64>::SMEM_BYTES);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128, true>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_bwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdTraits<128>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_bwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdTraits<64>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, F32Traits<128>::SMEM_BYTES);
@@ -149,6 +153,20 @@ int encode_map_packed(CUtensorMap* map, const void* base, int d, int H, long lon
     cuuint32_t box[3] = {64, 1, 128};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FATTN_OK : FATTN_ERR_CUDA;
+}
+
+// An 8-bit [outer, rows, inner] tensor (row pitch `pitch` bytes) in
+// 128-byte x 128-row boxes with 128-byte swizzle: the FP8 Q, K (inner = d)
+// and transposed V (inner = keys) tiles.
+int encode_map_u8(CUtensorMap* map, const void* base, long long inner, long long rows, long long outer, long long pitch) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(outer)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(pitch), static_cast<cuuint64_t>(pitch) * rows};
+    cuuint32_t box[3] = {128, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FATTN_OK : FATTN_ERR_CUDA;
@@ -353,6 +371,56 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     return cudaGetLastError() == cudaSuccess ? FATTN_OK : FATTN_ERR_CUDA;
 }
 
+int fp8_ld(int Lk) { return (Lk + 15) / 16 * 16; }
+
+int launch_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* qd, const float* kd, const float* vd,
+                   void* o, float* lse, int B, int H, int Lq, int Lk, int d, float scale, int causal, int wl, int wr,
+                   unsigned long long* visited, void* stream) {
+    int st = check_prefill(q8, k8, vt8, o, lse, B, H, Lq, Lk, d, scale);
+    if (st != FATTN_OK) return st;
+    if (!qd || !kd || !vd) return FATTN_ERR_INVALID_ARG;
+    if (d != 128) return FATTN_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(qd) | reinterpret_cast<uintptr_t>(kd) | reinterpret_cast<uintptr_t>(vd)) & 3u)
+        return FATTN_ERR_MISALIGNED;
+    DeviceInfo di;
+    st = device_ready(&di);
+    if (st != FATTN_OK) return st;
+    if (!di.fwd_regs_ok) return FATTN_ERR_UNSUPPORTED;
+    const long long BH = static_cast<long long>(B) * H;
+    const long long n_qtiles = (Lq + 127) / 128;
+    const long long n_pairs = (n_qtiles + 1) / 2;
+    const long long n_items = BH * n_pairs;
+    if (n_items > 0x7fffffffLL) return FATTN_ERR_UNSUPPORTED;
+    CUtensorMap mq, mk, mv;
+    if (encode_map_u8(&mq, q8, d, Lq, BH, d) != FATTN_OK || encode_map_u8(&mk, k8, d, Lk, BH, d) != FATTN_OK ||
+        encode_map_u8(&mv, vt8, Lk, d, BH, fp8_ld(Lk)) != FATTN_OK)
+        return FATTN_ERR_CUDA;
+    FwdParams p;
+    p.o = o;
+    p.lse = lse;
+    p.visited = visited;
+    p.B = B;
+    p.H = H;
+    p.Lq = Lq;
+    p.Lk = Lk;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.window_left = wl < 0 ? -1 : wl;
+    p.window_right = wr < 0 ? -1 : wr;
+    p.n_pairs = static_cast<int>(n_pairs);
+    p.n_items = static_cast<int>(n_items);
+    p.inject_stall = 0;
+    p.cu_q = p.cu_k = nullptr;
+    p.total_q = p.total_k = 0;
+    p.q_descale = qd;
+    p.k_descale = kd;
+    p.v_descale = vd;
+    const int grid = static_cast<int>(n_items < di.num_sms ? n_items : di.num_sms);
+    attn_fwd_sm100_kernel<128, false, true><<<grid, FwdTraits<128, true>::THREADS, FwdTraits<128, true>::SMEM_BYTES,
+                                               static_cast<cudaStream_t>(stream)>>>(mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? FATTN_OK : FATTN_ERR_CUDA;
+}
+
 int auto_splits(int B, int H, int Lk) {
     (void)B;
     (void)H;
@@ -541,6 +609,62 @@ int attn_count_blocks(int Lq, int Lk, int causal, int window_left, int window_ri
     if (partial) *partial = n_partial;
     if (pairs) *pairs = n_pairs;
     return FATTN_OK;
+}
+
+int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* q_descale, const float* k_descale,
+                 const float* v_descale, void* o, float* lse, int B, int H, int Lq, int Lk, int d, float scale, int causal,
+                 int window_left, int window_right, void* stream) {
+    return launch_fwd_fp8(q8, k8, vt8, q_descale, k_descale, v_descale, o, lse, B, H, Lq, Lk, d, scale, causal,
+                          window_left, window_right, nullptr, stream);
+}
+
+int attn_fwd_fp8_counted(const void* q8, const void* k8, const void* vt8, const float* q_descale,
+                         const float* k_descale, const float* v_descale, void* o, float* lse, int B, int H, int Lq,
+                         int Lk, int d, float scale, int causal, int window_left, int window_right,
+                         unsigned long long* kv_tiles_visited, void* stream) {
+    if (!kv_tiles_visited) return FATTN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(kv_tiles_visited) & 7u) return FATTN_ERR_MISALIGNED;
+    return launch_fwd_fp8(q8, k8, vt8, q_descale, k_descale, v_descale, o, lse, B, H, Lq, Lk, d, scale, causal,
+                          window_left, window_right, kv_tiles_visited, stream);
+}
+
+int attn_fp8_ld(int Lk) { return Lk < 1 ? 0 : fp8_ld(Lk); }
+
+int attn_quantize_fp8(const void* x, void* codes, float* descale, int B, int H, int L, int d, int transpose,
+                      void* stream) {
+    if (!x || !codes || !descale) return FATTN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || L < 1) return FATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FATTN_ERR_UNSUPPORTED;
+    const long long groups = static_cast<long long>(B) * H;
+    if (groups > 65535 || L > 0x7fffff00) return FATTN_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(descale) & 3u)) return FATTN_ERR_MISALIGNED;
+    DeviceInfo di;
+    int st = device_ready(&di);
+    if (st != FATTN_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto* bits = reinterpret_cast<unsigned int*>(descale);
+    const auto* xb = static_cast<const __nv_bfloat16*>(x);
+    auto* cb = static_cast<uint8_t*>(codes);
+    const long long group_len = static_cast<long long>(L) * d;
+    if (cudaMemsetAsync(descale, 0, static_cast<size_t>(groups) * sizeof(float), s) != cudaSuccess) {
+        cudaGetLastError();
+        return FATTN_ERR_CUDA;
+    }
+    long long per_group = (group_len / 8 + 255) / 256;
+    const unsigned bx = static_cast<unsigned>(per_group < 64 ? per_group : 64);
+    fp8_amax_kernel<<<dim3(bx, static_cast<unsigned>(groups)), 256, 0, s>>>(xb, bits, group_len);
+    if (transpose) {
+        const int ld = fp8_ld(L);
+        const dim3 grid(static_cast<unsigned>((ld + 63) / 64), static_cast<unsigned>(groups));
+        if (d == 128)
+            fp8_quant_t_kernel<128><<<grid, 256, 0, s>>>(xb, bits, cb, L, ld);
+        else
+            fp8_quant_t_kernel<64><<<grid, 256, 0, s>>>(xb, bits, cb, L, ld);
+    } else {
+        fp8_quant_kernel<<<dim3(bx, static_cast<unsigned>(groups)), 256, 0, s>>>(xb, bits, cb, group_len);
+    }
+    fp8_descale_kernel<<<static_cast<unsigned>((groups + 255) / 256), 256, 0, s>>>(bits, static_cast<int>(groups));
+    return cudaGetLastError() == cudaSuccess ? FATTN_OK : FATTN_ERR_CUDA;
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int Lq, int d) {

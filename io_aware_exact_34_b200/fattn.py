@@ -53,6 +53,15 @@ lib.attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i]
 lib.attn_bwd_workspace_bytes.restype = _sz
 lib.attn_bwd_count_blocks.argtypes = [_i, _i, _i, _i, _i, _i, _i, _llp]
 lib.attn_bwd_count_blocks.restype = _i
+lib.attn_fwd_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp]
+lib.attn_fwd_fp8.restype = _i
+lib.attn_fwd_fp8_counted.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp,
+                                     _vp]
+lib.attn_fwd_fp8_counted.restype = _i
+lib.attn_fp8_ld.argtypes = [_i]
+lib.attn_fp8_ld.restype = _i
+lib.attn_quantize_fp8.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
+lib.attn_quantize_fp8.restype = _i
 lib.fattn_status_string.argtypes = [_i]
 lib.fattn_status_string.restype = ctypes.c_char_p
 lib.fattn_device_status.argtypes = [_vp]
@@ -258,6 +267,51 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seqlens_k, o=None, lse=N
     _check(lib.attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), max_pages, page_size,
                                  num_pages, _ptr(o), _ptr(lse), _ptr(seqlens_k), B, H, d, scale, S, _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream()), "attn_decode_paged")
+    return o, lse
+
+
+def attn_fp8_ld(Lk) -> int:
+    return lib.attn_fp8_ld(Lk)
+
+
+def attn_quantize_fp8(x, transpose=False, codes=None, descale=None):
+    """bf16 [B,H,L,d] -> (e4m3 codes as uint8 [B,H,L,d], or [B,H,d,ld] when
+    transposed; fp32 descale [B,H])."""
+    _want(x, torch.bfloat16, 4, "x")
+    B, H, L, d = x.shape
+    if codes is None:
+        shape = (B, H, d, attn_fp8_ld(L)) if transpose else (B, H, L, d)
+        codes = torch.empty(shape, dtype=torch.uint8, device=x.device)
+    if descale is None:
+        descale = torch.empty((B, H), dtype=torch.float32, device=x.device)
+    _check(lib.attn_quantize_fp8(_ptr(x), _ptr(codes), _ptr(descale), B, H, L, d, int(bool(transpose)), _stream()),
+           "attn_quantize_fp8")
+    return codes, descale
+
+
+def attn_fwd_fp8(q8, k8, vt8, q_descale, k_descale, v_descale, o=None, lse=None, scale=None, causal=False,
+                 window_left=-1, window_right=-1, counter=None):
+    """FP8 prefill forward.  q8: [B,H,Lq,128], k8: [B,H,Lk,128] and vt8:
+    [B,H,128,ld] uint8 e4m3 codes; descales fp32 [B,H] -> (o bf16, lse fp32)."""
+    for t, name in ((q8, "q8"), (k8, "k8"), (vt8, "vt8")):
+        _want(t, torch.uint8, 4, name)
+    for t, name in ((q_descale, "q_descale"), (k_descale, "k_descale"), (v_descale, "v_descale")):
+        _want(t, torch.float32, 2, name)
+    B, H, Lq, d = q8.shape
+    Lk = k8.shape[2]
+    if tuple(vt8.shape) != (B, H, d, attn_fp8_ld(Lk)):
+        raise ValueError(f"vt8: expected shape {(B, H, d, attn_fp8_ld(Lk))}, got {tuple(vt8.shape)}")
+    if o is None:
+        o = torch.empty((B, H, Lq, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q8.device)
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    args = (_ptr(q8), _ptr(k8), _ptr(vt8), _ptr(q_descale), _ptr(k_descale), _ptr(v_descale), _ptr(o), _ptr(lse),
+            B, H, Lq, Lk, d, scale, int(bool(causal)), int(window_left), int(window_right))
+    if counter is None:
+        _check(lib.attn_fwd_fp8(*args, _stream()), "attn_fwd_fp8")
+    else:
+        _check(lib.attn_fwd_fp8_counted(*args, _ptr(counter), _stream()), "attn_fwd_fp8_counted")
     return o, lse
 
 

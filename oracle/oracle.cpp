@@ -132,11 +132,16 @@ double e4m3_value(uint8_t code) {
  * over the 127 finite non-negative codes. */
 uint8_t e4m3_round(double x) {
     if (std::isnan(x)) return 0x7F;
+    static const std::vector<double> table = [] {
+        std::vector<double> t(0x7F);
+        for (int c = 0; c <= 0x7E; ++c) t[c] = e4m3_value(static_cast<uint8_t>(c));
+        return t;
+    }();
     const double a = std::fabs(x);
     int best = 0;
     double best_d = std::numeric_limits<double>::infinity();
     for (int c = 0; c <= 0x7E; ++c) {
-        const double d = std::fabs(e4m3_value(static_cast<uint8_t>(c)) - a);
+        const double d = std::fabs(table[c] - a);
         if (d < best_d || (d == best_d && (c & 1) == 0)) {
             best = c;
             best_d = d;

@@ -221,3 +221,22 @@ def test_bwd_scheduler_matches_bruteforce(fl, oracle, Lq, Lk, causal, wl, wr, bq
     exactly the tiles with an allowed pair: the oracle's brute-force count."""
     got = fl.attn_bwd_count_blocks(Lq, Lk, causal, wl, wr, bq, bk)
     assert got == oracle.count_blocks(Lq, Lk, causal, wl, wr, bq, bk)["visited"]
+
+
+def test_fp8_argument_checks(fl):
+    def fwd(d=128, qd=FAKE, kd=FAKE, vd=FAKE, q=FAKE, Lk=300):
+        return fl.lib.attn_fwd_fp8(q, FAKE, FAKE, qd, kd, vd, FAKE, None, 1, 2, 300, Lk, d, 0.1, 1, -1, -1, None)
+    assert fwd(d=64) == fl.FATTN_ERR_UNSUPPORTED
+    assert fwd(qd=None) == fl.FATTN_ERR_INVALID_ARG
+    assert fwd(vd=FAKE + 2) == fl.FATTN_ERR_MISALIGNED
+    assert fwd(q=FAKE + 8) == fl.FATTN_ERR_MISALIGNED
+    assert fwd(Lk=0) == fl.FATTN_ERR_INVALID_ARG
+    assert [fl.attn_fp8_ld(n) for n in (1, 16, 17, 300, 4096, 0)] == [16, 16, 32, 304, 4096, 0]
+    q = fl.lib.attn_quantize_fp8
+    assert q(FAKE, FAKE, FAKE, 1, 1, 10, 96, 0, None) == fl.FATTN_ERR_UNSUPPORTED
+    assert q(None, FAKE, FAKE, 1, 1, 10, 128, 0, None) == fl.FATTN_ERR_INVALID_ARG
+    assert q(FAKE, FAKE, FAKE + 2, 1, 1, 10, 128, 0, None) == fl.FATTN_ERR_MISALIGNED
+    assert q(FAKE, FAKE, FAKE, 1, 70000, 10, 128, 0, None) == fl.FATTN_ERR_UNSUPPORTED
+    if not torch.cuda.is_available():
+        assert fwd() == fl.FATTN_ERR_NO_DEVICE
+        assert q(FAKE, FAKE, FAKE, 1, 1, 10, 128, 1, None) == fl.FATTN_ERR_NO_DEVICE
