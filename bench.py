@@ -54,6 +54,7 @@ KERNEL_SOURCES = {
     "attn_fwd_sm100_kernel": ["attn_fwd_sm100.cuh", "sched.cuh", "dev_prims.cuh"],
     "decode_split_kernel": ["decode_splitkv.cuh", "dev_prims.cuh"],
     "attn_bwd_sm100_kernel": ["attn_bwd_sm100.cuh", "sched.cuh", "dev_prims.cuh"],
+    "attn_fwd_fp8": ["attn_fwd_sm100.cuh", "sched.cuh", "dev_prims.cuh"],
 }
 
 
@@ -384,7 +385,7 @@ def run_ours(args, world, rank, local):
         fp8 = {"metric": "attention fwd TFLOP/s (in-mask FLOPs), e4m3 Q/K/V/P", "value": world * tf,
                "unit": "TFLOP/s", "ms_per_step": fms, "steps": fsteps,
                "roofline": {"bound": "tensor", "achieved": tf, "peak": fp8_peak, "unit": "TFLOP/s",
-                            "frac": tf / fp8_peak, "traffic": None,
+                            "frac": tf / fp8_peak, "traffic": recorded_traffic("attn_fwd_fp8", w.name),
                             "peak_source": f"{peak_src} bf16 dense (burst) x 2 (nominal fp8/bf16 ratio)",
                             "kernel": PREFILL_KERNEL + "<128, false, true>"},
                "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
