@@ -28,14 +28,16 @@
 //
 // Main kernel, 512 threads:
 //   warp 0       TMA producer: K_j and V_j once, then a 2-stage ring of
-//                (Q_i, dO_i, LSE_i, D_i)
+//                (Q_i, LSE_i, D_i) and dO_i, each half with its own barriers
 //   warp 1       MMA issuer (one thread)
 //   warps 4-11   two warpgroups, thread = key row; warpgroup h owns the query
 //                columns [64h, 64h+64) of every score tile: P, dS
 //   warps 12-15  dQ drain, thread = query row: the dQ tile goes from tensor
 //                memory into the stage buffer its Q and dO tiles have left
 //                (the fp32 128 x D tile is exactly their size), then TMA
-//                reduce-adds it into the fp32 accumulator in whole lines
+//                reduce-adds it into the fp32 accumulator in whole lines;
+//                the Q half is released as soon as its boxes have been read,
+//                so the next Q tile can load while the dO half still drains
 //
 // Tensor memory (512 columns), lane = key row unless noted:
 //   [0,128)        S^T = K_j Q_i^T (fp32), then P^T (bf16 pairs) over it
@@ -76,6 +78,9 @@ __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bul
 // Until every committed bulk operation of this thread has read its shared-memory source.
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
+// Until at most the most recent committed bulk group of this thread is still reading its source.
+__device__ __forceinline__ void bulk_wait_read_one() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+
 // Until every committed bulk operation of this thread has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -95,7 +100,7 @@ struct BwdTraits {
     static constexpr int SMEM_VEC_OFF = SMEM_DS_OFF + DS_BYTES;  // stage s: LSE2 at +0, D at +512
     static constexpr int VEC_STAGE_BYTES = 1024;
     static constexpr int SMEM_BAR_OFF = SMEM_VEC_OFF + NSTAGE * VEC_STAGE_BYTES;
-    static constexpr int NBAR = 1 + 2 * NSTAGE + 9;
+    static constexpr int NBAR = 1 + 4 * NSTAGE + 9;
     static constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NBAR * 8;
     static constexpr int SMEM_USED = SMEM_MISC_OFF + 16;
     // Alignment slack for the 1024-byte aligned base; the kernel checks at run
@@ -243,9 +248,11 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t sVec = base + T::SMEM_VEC_OFF;
     const uint32_t bar0 = base + T::SMEM_BAR_OFF;
     const uint32_t kv_full = bar0;
-    const uint32_t qd_full0 = bar0 + 8;
-    const uint32_t qd_empty0 = qd_full0 + 8 * T::NSTAGE;
-    const uint32_t s_full = qd_empty0 + 8 * T::NSTAGE;
+    const uint32_t q_full0 = bar0 + 8;                   // Q + LSE2 + D of a stage landed
+    const uint32_t do_full0 = q_full0 + 8 * T::NSTAGE;   // dO of a stage landed
+    const uint32_t q_empty0 = do_full0 + 8 * T::NSTAGE;  // Q half of a stage free
+    const uint32_t do_empty0 = q_empty0 + 8 * T::NSTAGE; // dO half of a stage free
+    const uint32_t s_full = do_empty0 + 8 * T::NSTAGE;
     const uint32_t dp_full = s_full + 8;
     const uint32_t p_ready = dp_full + 8;
     const uint32_t ds_ready = p_ready + 8;
@@ -264,8 +271,11 @@ __global__ void __launch_bounds__(512, 1)
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
         for (int s = 0; s < T::NSTAGE; ++s) {
-            mbar_init(qd_full0 + 8 * s, 1);
-            mbar_init(qd_empty0 + 8 * s, 2);  // the MMA warp's commit and the dQ drain's release
+            mbar_init(q_full0 + 8 * s, 1);
+            mbar_init(do_full0 + 8 * s, 1);
+            // the MMA warp's commit and the dQ drain's release
+            mbar_init(q_empty0 + 8 * s, 2);
+            mbar_init(do_empty0 + 8 * s, 2);
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
@@ -304,33 +314,44 @@ __global__ void __launch_bounds__(512, 1)
                 tma_load_3d(sV + c * T::CHUNK_BYTES, &tm_v, kv_full, c * 64, static_cast<int>(tile.k0), tile.bh);
             }
             bool ok = true;
-            int issued = 0;
+            int issued = 0, issued_do = 0;
             for (int n = 0; n < n_tiles && ok; ++n) {
                 const int s = n & 1;
                 const uint32_t use = static_cast<uint32_t>(n >> 1);
+                const int q0 = (tile.q_lo + n) * 128;
+                const uint32_t st = sStage + s * 2 * T::TILE_BYTES;
                 if (use > 0) {
-                    ok = mbar_wait(qd_empty0 + 8 * s, (use - 1) & 1u, abort_flag, status, -6);
+                    ok = mbar_wait(q_empty0 + 8 * s, (use - 1) & 1u, abort_flag, status, -6);
                     if (!ok) break;
                 }
-                const int q0 = (tile.q_lo + n) * 128;
-                const uint32_t fb = qd_full0 + 8 * s;
-                const uint32_t st = sStage + s * 2 * T::TILE_BYTES;
-                mbar_arrive_expect_tx(fb, 2 * T::TILE_BYTES + T::VEC_STAGE_BYTES);
-                for (int c = 0; c < T::NCHUNK; ++c) {
-                    tma_load_3d(st + c * T::CHUNK_BYTES, &tm_q, fb, c * 64, q0, tile.bh);
-                    tma_load_3d(st + T::TILE_BYTES + c * T::CHUNK_BYTES, &tm_do, fb, c * 64, q0, tile.bh);
-                }
+                const uint32_t qfb = q_full0 + 8 * s;
+                mbar_arrive_expect_tx(qfb, T::TILE_BYTES + T::VEC_STAGE_BYTES);
+                for (int c = 0; c < T::NCHUNK; ++c)
+                    tma_load_3d(st + c * T::CHUNK_BYTES, &tm_q, qfb, c * 64, q0, tile.bh);
                 const long long voff = static_cast<long long>(tile.bh) * p.Lq_pad + q0;
-                bulk_load(sVec + s * T::VEC_STAGE_BYTES, p.lse2 + voff, 512, fb);
-                bulk_load(sVec + s * T::VEC_STAGE_BYTES + 512, p.dsum + voff, 512, fb);
+                bulk_load(sVec + s * T::VEC_STAGE_BYTES, p.lse2 + voff, 512, qfb);
+                bulk_load(sVec + s * T::VEC_STAGE_BYTES + 512, p.dsum + voff, 512, qfb);
                 ++issued;
+                if (use > 0) {
+                    ok = mbar_wait(do_empty0 + 8 * s, (use - 1) & 1u, abort_flag, status, -6);
+                    if (!ok) break;
+                }
+                const uint32_t dfb = do_full0 + 8 * s;
+                mbar_arrive_expect_tx(dfb, T::TILE_BYTES);
+                for (int c = 0; c < T::NCHUNK; ++c)
+                    tma_load_3d(st + T::TILE_BYTES + c * T::CHUNK_BYTES, &tm_do, dfb, c * 64, q0, tile.bh);
+                ++issued_do;
             }
             // No copy may still be landing in shared memory when the CTA exits.
             mbar_wait(kv_full, 0, nullptr, status, -6);
             for (int s = 0; s < T::NSTAGE; ++s) {
                 if (issued > s) {
                     const uint32_t uses = static_cast<uint32_t>((issued - 1 - s) / T::NSTAGE + 1);
-                    mbar_wait(qd_full0 + 8 * s, (uses - 1) & 1u, nullptr, status, -6);
+                    mbar_wait(q_full0 + 8 * s, (uses - 1) & 1u, nullptr, status, -6);
+                }
+                if (issued_do > s) {
+                    const uint32_t uses = static_cast<uint32_t>((issued_do - 1 - s) / T::NSTAGE + 1);
+                    mbar_wait(do_full0 + 8 * s, (uses - 1) & 1u, nullptr, status, -6);
                 }
             }
         }
@@ -354,7 +375,7 @@ __global__ void __launch_bounds__(512, 1)
                 }
                 mma_commit(s_full);
             };
-            if (ok) ok = mbar_wait(qd_full0, 0, abort_flag, status, -6);
+            if (ok) ok = mbar_wait(q_full0, 0, abort_flag, status, -6);
             if (ok) {
                 tc_fence_after_sync();
                 issue_s(0);
@@ -369,6 +390,9 @@ __global__ void __launch_bounds__(512, 1)
                     if (!ok) break;
                     tc_fence_after_sync();
                 }
+                ok = mbar_wait(do_full0 + 8 * s, static_cast<uint32_t>(n >> 1) & 1u, abort_flag, status, -6);
+                if (!ok) break;
+                tc_fence_after_sync();
                 {
                     const uint32_t d_lo = sdesc_lo(do_st, 16);
                     const uint32_t v_lo = sdesc_lo(sV, 16);
@@ -393,10 +417,11 @@ __global__ void __launch_bounds__(512, 1)
                                     idesc_g, (n > 0 || ks > 0) ? 1u : 0u);
                     }
                 }
+                mma_commit(do_empty0 + 8 * s);  // dV(n) was the last product to read dO(n)
                 // the next tile's scores go in now that P^T has been issued to its consumer
                 if (n + 1 < n_tiles) {
                     const int s1 = (n + 1) & 1;
-                    ok = mbar_wait(qd_full0 + 8 * s1, static_cast<uint32_t>((n + 1) >> 1) & 1u, abort_flag, status, -6);
+                    ok = mbar_wait(q_full0 + 8 * s1, static_cast<uint32_t>((n + 1) >> 1) & 1u, abort_flag, status, -6);
                     if (!ok) break;
                     tc_fence_after_sync();
                     issue_s(n + 1);
@@ -425,7 +450,7 @@ __global__ void __launch_bounds__(512, 1)
                                     sdesc_from_lo(b_lo + ks * (2048 >> 4)), idesc_q, ks > 0 ? 1u : 0u);
                 }
                 mma_commit(dq_full);
-                mma_commit(qd_empty0 + 8 * s);
+                mma_commit(q_empty0 + 8 * s);
             }
             if (ok) mma_commit(dkdv_full);
         }
@@ -607,12 +632,18 @@ __global__ void __launch_bounds__(512, 1)
             if (leader) {
                 ok = mbar_wait(dq_staged, n & 1u, abort_flag, status, -6);
                 if (ok) {
+                    // boxes [0, D/64) sit in the Q half of the stage, the rest in the dO half
                     const int y = tile.bh * p.Lq_pad + (tile.q_lo + n) * 128;
-                    for (int ch = 0; ch < D / 32; ++ch)
+                    for (int ch = 0; ch < D / 64; ++ch)
                         tma_reduce_add_2d(&tm_dq, smem_addr(stage) + ch * 16384, ch * 32, y);
                     bulk_commit_group();
+                    for (int ch = D / 64; ch < D / 32; ++ch)
+                        tma_reduce_add_2d(&tm_dq, smem_addr(stage) + ch * 16384, ch * 32, y);
+                    bulk_commit_group();
+                    bulk_wait_read_one();
+                    mbar_arrive(q_empty0 + 8 * s);   // the Q half may be refilled
                     bulk_wait_read_all();
-                    mbar_arrive(qd_empty0 + 8 * s);  // the stage buffer may be refilled
+                    mbar_arrive(do_empty0 + 8 * s);  // and the dO half
                 }
             }
             __syncwarp();
