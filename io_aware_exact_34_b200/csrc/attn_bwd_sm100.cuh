@@ -32,12 +32,12 @@
 //   warp 1       MMA issuer (one thread)
 //   warps 4-11   two warpgroups, thread = key row; warpgroup h owns the query
 //                columns [64h, 64h+64) of every score tile: P, dS
-//   warps 12-15  dQ drain, thread = query row: the dQ tile goes from tensor
-//                memory into the stage buffer its Q and dO tiles have left
-//                (the fp32 128 x D tile is exactly their size), then TMA
-//                reduce-adds it into the fp32 accumulator in whole lines;
-//                the Q half is released as soon as its boxes have been read,
-//                so the next Q tile can load while the dO half still drains
+//   warps 12-15  dQ drain, thread = query row: the dQ tile leaves tensor
+//                memory in two halves of D/2 columns, each staged in the dO
+//                buffer of its stage (free once dV has read dO; 128 x D/2
+//                fp32 is exactly its size) and TMA reduce-added into the fp32
+//                accumulator in whole lines; the Q buffer is never used for
+//                it, so the next Q tile loads as soon as dK has read the last
 //
 // Tensor memory (512 columns), lane = key row unless noted:
 //   [0,128)        S^T = K_j Q_i^T (fp32), then P^T (bf16 pairs) over it
@@ -73,6 +73,16 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32
                  : "memory");
 }
 
+__device__ __forceinline__ float4 lds128(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Until every committed bulk operation of this thread has read its shared-memory source.
@@ -100,7 +110,7 @@ struct BwdTraits {
     static constexpr int SMEM_VEC_OFF = SMEM_DS_OFF + DS_BYTES;  // stage s: LSE2 at +0, D at +512
     static constexpr int VEC_STAGE_BYTES = 1024;
     static constexpr int SMEM_BAR_OFF = SMEM_VEC_OFF + NSTAGE * VEC_STAGE_BYTES;
-    static constexpr int NBAR = 1 + 4 * NSTAGE + 9;
+    static constexpr int NBAR = 1 + 4 * NSTAGE + 10;
     static constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NBAR * 8;
     static constexpr int SMEM_USED = SMEM_MISC_OFF + 16;
     // Alignment slack for the 1024-byte aligned base; the kernel checks at run
@@ -111,8 +121,8 @@ struct BwdTraits {
     static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(SMEM_USED <= 232448, "shared memory");
-    // the dQ tile (128 x D fp32) is staged in a stage buffer (Q + dO, 128 x D bf16 each)
-    static_assert(128 * D * 4 == 2 * TILE_BYTES, "dQ staging");
+    // half a dQ tile (128 x D/2 fp32) is staged in a dO buffer (128 x D bf16)
+    static_assert(128 * (D / 2) * 4 == TILE_BYTES, "dQ staging");
 };
 
 struct BwdParams {
@@ -261,6 +271,7 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t dkdv_full = dq_empty + 8;
     const uint32_t drain_bar = dkdv_full + 8;
     const uint32_t dq_staged = drain_bar + 8;
+    const uint32_t stage_reuse = dq_staged + 8;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + T::SMEM_MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + T::SMEM_MISC_OFF + 4);
 
@@ -273,9 +284,8 @@ __global__ void __launch_bounds__(512, 1)
         for (int s = 0; s < T::NSTAGE; ++s) {
             mbar_init(q_full0 + 8 * s, 1);
             mbar_init(do_full0 + 8 * s, 1);
-            // the MMA warp's commit and the dQ drain's release
-            mbar_init(q_empty0 + 8 * s, 2);
-            mbar_init(do_empty0 + 8 * s, 2);
+            mbar_init(q_empty0 + 8 * s, 1);   // the MMA warp's commit after dK
+            mbar_init(do_empty0 + 8 * s, 2);  // the MMA warp's commit after dV and the dQ drain's release
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
@@ -286,6 +296,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(dkdv_full, 1);
         mbar_init(drain_bar, 1);
         mbar_init(dq_staged, 128);
+        mbar_init(stage_reuse, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -439,6 +450,7 @@ __global__ void __launch_bounds__(512, 1)
                                     idesc_g, (n > 0 || ks > 0) ? 1u : 0u);
                     }
                 }
+                mma_commit(q_empty0 + 8 * s);  // dK(n) was the last product to read Q(n)
                 // dQ = dS K into [128,256): A = dS (shared memory, query-contiguous rows
                 // per key), B = K (key rows, MN-major over d); 16 keys per step
                 {
@@ -450,7 +462,6 @@ __global__ void __launch_bounds__(512, 1)
                                     sdesc_from_lo(b_lo + ks * (2048 >> 4)), idesc_q, ks > 0 ? 1u : 0u);
                 }
                 mma_commit(dq_full);
-                mma_commit(q_empty0 + 8 * s);
             }
             if (ok) mma_commit(dkdv_full);
         }
@@ -477,7 +488,8 @@ __global__ void __launch_bounds__(512, 1)
             const bool full = q0 + 127 <= p.Lq - 1 && tile_is_full(band, q0, q0 + 127, tile.k0, 128);
             const int c_lo = clamp_int(i_lo - q0) - 64 * h;  // relative to this half's first column
             const int c_hi = clamp_int(i_hi - q0) - 64 * h;
-            const float* vec = reinterpret_cast<const float*>(gbase + T::SMEM_VEC_OFF + s * T::VEC_STAGE_BYTES) + 64 * h;
+            // LSE2 of this half's 64 query columns at vec, D at vec + 512 (shared addresses)
+            const uint32_t vec = sVec + s * T::VEC_STAGE_BYTES + 64 * h * 4;
             // P = exp2(s * scale * log2(e) - LSE2), zero where masked
             ok = mbar_wait(s_full, n & 1u, abort_flag, status, -6);
             ok = __all_sync(0xffffffffu, ok);
@@ -490,10 +502,10 @@ __global__ void __launch_bounds__(512, 1)
                 tmem_ld32(tmem + lane_off + T::TM_S + 64 * h + 32 * cc, sr);
                 tmem_wait_ld();
                 reg_fence(sr);
-                const float4* l4 = reinterpret_cast<const float4*>(vec + 32 * cc);
+
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 l = l4[e4];
+                    const float4 l = lds128(vec + (32 * cc + 4 * e4) * 4);
                     const float ls[4] = {l.x, l.y, l.z, l.w};
                     float pv[4];
 #pragma unroll
@@ -523,10 +535,10 @@ __global__ void __launch_bounds__(512, 1)
                 tmem_ld32(tmem + lane_off + T::TM_DP + 64 * h + 32 * cc, dr);
                 tmem_wait_ld();
                 reg_fence(dr);
-                const float4* d4 = reinterpret_cast<const float4*>(vec + 128 + 32 * cc);
+
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 dd = d4[e4];
+                    const float4 dd = lds128(vec + 512 + (32 * cc + 4 * e4) * 4);
                     const float ds[4] = {dd.x, dd.y, dd.z, dd.w};
                     float g[4];
 #pragma unroll
@@ -543,11 +555,10 @@ __global__ void __launch_bounds__(512, 1)
             // dS into shared memory as row `row` (key) of the [key][query] operand:
             // 64 queries = one 128-byte row of swizzle column h, 16-byte unit u at u ^ (row & 7)
             {
-                uint8_t* drow = gbase + T::SMEM_DS_OFF + h * 16384 + row * 128;
+                const uint32_t drow = sDS + h * 16384 + row * 128;
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
-                    *reinterpret_cast<uint4*>(drow + ((u ^ (row & 7)) << 4)) =
-                        make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+                    sts128(drow + ((u ^ (row & 7)) << 4), dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
             }
             fence_proxy_async_smem();
             tmem_wait_st();
@@ -595,10 +606,31 @@ __global__ void __launch_bounds__(512, 1)
             atomicAdd(p.visited, static_cast<unsigned long long>(n_tiles));
     } else if (warp >= 12) {
         // ------------------------------------------------------------ dQ drain
+        constexpr int NB = D / 64;  // 32-column boxes per half tile
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;  // query row of the dQ tile
         const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + T::TM_DP;
         const bool leader = warp == 12 && lane == 0;
+        // one half tile (NB boxes of 32 columns, 128-byte rows, 128-byte swizzle) into buf
+        auto stage_half = [&](uint32_t buf, uint32_t (&r)[NB][32]) {
+#pragma unroll
+            for (int c = 0; c < NB; ++c)
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    sts128(buf + c * 16384 + row * 128 + ((u ^ (row & 7)) << 4), r[c][4 * u], r[c][4 * u + 1],
+                           r[c][4 * u + 2], r[c][4 * u + 3]);
+            fence_proxy_async_smem();
+            mbar_arrive(dq_staged);
+        };
+        // leader: reduce-add the staged half once all 128 rows are in, wait until it is read
+        auto reduce_half = [&](uint32_t buf, int col0, int y, uint32_t parity, uint32_t release) -> bool {
+            if (!mbar_wait(dq_staged, parity, abort_flag, status, -6)) return false;
+            for (int c = 0; c < NB; ++c) tma_reduce_add_2d(&tm_dq, buf + c * 16384, col0 + 32 * c, y);
+            bulk_commit_group();
+            bulk_wait_read_all();
+            mbar_arrive(release);
+            return true;
+        };
         bool ok = true;
         for (int n = 0; n < n_tiles && ok; ++n) {
             const int s = n & 1;
@@ -606,46 +638,31 @@ __global__ void __launch_bounds__(512, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after_sync();
-            // dQ(n) has completed, so every MMA that read this stage's Q and dO
-            // tiles has too: the stage buffer takes the fp32 tile, 32 columns
-            // (16 KB, 128-byte rows, 128-byte swizzle) per TMA box
-            uint8_t* stage = gbase + T::SMEM_STAGE_OFF + s * 2 * T::TILE_BYTES;
-#pragma unroll 1
-            for (int ch = 0; ch < D / 32; ++ch) {
-                uint32_t r[32];
-                tmem_ld32(taddr + ch * 32, r);
-                tmem_wait_ld();
-                reg_fence(r);
-                if (ch == D / 32 - 1) {
-                    // the whole tile is in registers or shared memory: release tensor memory
-                    tc_fence_before_sync();
-                    mbar_arrive(dq_empty);
-                }
-                uint8_t* dst = stage + ch * 16384 + row * 128;
+            // dQ(n) has completed, so dV(n) has read dO(n): its buffer takes the halves
+            const uint32_t buf = sStage + s * 2 * T::TILE_BYTES + T::TILE_BYTES;
+            const int y = tile.bh * p.Lq_pad + (tile.q_lo + n) * 128;
+            uint32_t r[NB][32];
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    *reinterpret_cast<uint4*>(dst + ((u ^ (row & 7)) << 4)) =
-                        make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(dq_staged);
-            if (leader) {
-                ok = mbar_wait(dq_staged, n & 1u, abort_flag, status, -6);
-                if (ok) {
-                    // boxes [0, D/64) sit in the Q half of the stage, the rest in the dO half
-                    const int y = tile.bh * p.Lq_pad + (tile.q_lo + n) * 128;
-                    for (int ch = 0; ch < D / 64; ++ch)
-                        tma_reduce_add_2d(&tm_dq, smem_addr(stage) + ch * 16384, ch * 32, y);
-                    bulk_commit_group();
-                    for (int ch = D / 64; ch < D / 32; ++ch)
-                        tma_reduce_add_2d(&tm_dq, smem_addr(stage) + ch * 16384, ch * 32, y);
-                    bulk_commit_group();
-                    bulk_wait_read_one();
-                    mbar_arrive(q_empty0 + 8 * s);   // the Q half may be refilled
-                    bulk_wait_read_all();
-                    mbar_arrive(do_empty0 + 8 * s);  // and the dO half
-                }
-            }
+            for (int c = 0; c < NB; ++c) tmem_ld32(taddr + 32 * c, r[c]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < NB; ++c) reg_fence(r[c]);
+            stage_half(buf, r);
+            // the second half goes to registers and tensor memory is released
+#pragma unroll
+            for (int c = 0; c < NB; ++c) tmem_ld32(taddr + D / 2 + 32 * c, r[c]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < NB; ++c) reg_fence(r[c]);
+            tc_fence_before_sync();
+            mbar_arrive(dq_empty);
+            if (leader) ok = reduce_half(buf, 0, y, 0u, stage_reuse);
+            __syncwarp();
+            ok = __all_sync(0xffffffffu, ok) && mbar_wait(stage_reuse, n & 1u, abort_flag, status, -6);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            stage_half(buf, r);
+            if (leader) ok = reduce_half(buf, D / 2, y, 1u, do_empty0 + 8 * s);
             __syncwarp();
             ok = __all_sync(0xffffffffu, ok);
         }
