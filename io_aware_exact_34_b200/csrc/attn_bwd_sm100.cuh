@@ -513,7 +513,8 @@ __global__ void __launch_bounds__(512, 1)
                         const int c = 32 * cc + 4 * e4 + u;
                         const float x = __uint_as_float(sr[4 * e4 + u]) * c_log2 - ls[u];
                         const bool allowed = full || (c >= c_lo && c <= c_hi);
-                        pv[u] = allowed ? fast_exp2(x) : 0.f;
+                        // masked: 2^-inf = 0; the exponential itself is never conditional
+                        pv[u] = fast_exp2(allowed ? x : -CUDART_INF_F);
                     }
                     pk[16 * cc + 2 * e4] = pack_bf16x2(pv[0], pv[1]);
                     pk[16 * cc + 2 * e4 + 1] = pack_bf16x2(pv[2], pv[3]);
