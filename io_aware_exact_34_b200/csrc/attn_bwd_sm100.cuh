@@ -88,9 +88,6 @@ __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bul
 // Until every committed bulk operation of this thread has read its shared-memory source.
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
-// Until at most the most recent committed bulk group of this thread is still reading its source.
-__device__ __forceinline__ void bulk_wait_read_one() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
-
 // Until every committed bulk operation of this thread has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 

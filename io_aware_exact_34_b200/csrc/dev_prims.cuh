@@ -202,21 +202,13 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int a_mn, in
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 layout version 1.
-// lbo / sbo: leading / stride byte offsets.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
-    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
-    d |= static_cast<uint64_t>(1) << 46;  // descriptor version
-    d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
-    return d;
-}
-
-// The same descriptor split into its words: the high word (stride byte
-// offset 1024, version 1, 128-byte swizzle) is shared by every operand here;
-// the low word carries the start address and the leading byte offset.
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 layout version 1:
+// start address >> 4 in bits 0-13, leading byte offset >> 4 in bits 16-29,
+// stride byte offset >> 4 in bits 32-45, version 1 at bit 46, layout 2
+// (128-byte swizzle) in bits 61-63.
+// The descriptor split into its words: the high word (stride byte offset
+// 1024, version 1, 128-byte swizzle) is shared by every operand here; the low
+// word carries the start address and the leading byte offset.
 constexpr uint32_t kSdescHiSw128Sbo1024 = (1024u >> 4) | (1u << 14) | (2u << 29);
 
 __device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo) {
@@ -309,12 +301,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
 

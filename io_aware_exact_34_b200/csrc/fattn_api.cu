@@ -506,7 +506,7 @@ int attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
     if (d != 64 && d != 128) return FATTN_ERR_UNSUPPORTED;
     if (B > 65535 || H > 65535 || Lk > 0x7fffff00) return FATTN_ERR_UNSUPPORTED;
     const int S = num_splits == 0 ? auto_splits(B, H, Lk) : num_splits;
-    if (S > Lk || S > 0x7fffffff / 1) return FATTN_ERR_INVALID_ARG;
+    if (S > Lk) return FATTN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return FATTN_ERR_MISALIGNED;
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FATTN_ERR_MISALIGNED;
     if (seqlens_k && (reinterpret_cast<uintptr_t>(seqlens_k) & 3u)) return FATTN_ERR_MISALIGNED;
