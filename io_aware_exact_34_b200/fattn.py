@@ -98,29 +98,61 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def _want(t, dtype, ndim, name):
+def _want(t, dtype, ndim, name, shape=None, device=None):
+    """Every pointer the library receives comes from a tensor checked here:
+    dtype, rank, contiguity, CUDA residency and, where given, the exact shape
+    and the device of the first input (the kernels trust all of these)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype or t.dim() != ndim or not t.is_cuda or not t.is_contiguous():
         raise ValueError(f"{name}: expected a contiguous {dtype} CUDA tensor with {ndim} dims, got "
                          f"{t.dtype} {tuple(t.shape)} on {t.device}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+
+
+def _want_counter(counter, device):
+    if counter is not None:
+        if not isinstance(counter, torch.Tensor) or counter.dtype not in (torch.int64, torch.uint64) \
+                or counter.numel() != 1 or not counter.is_cuda or counter.device != device:
+            raise ValueError(f"counter: expected a one-element int64 tensor on {device}")
+
+
+def _want_workspace(ws, device):
+    if ws is not None:
+        if not isinstance(ws, torch.Tensor) or not ws.is_cuda or ws.device != device or not ws.is_contiguous():
+            raise ValueError(f"workspace: expected a contiguous CUDA tensor on {device}")
 
 
 def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, window_left=-1, window_right=-1,
-             need_lse=True):
-    """bf16 prefill forward.  q: [B,H,Lq,d], k, v: [B,H,Lk,d] -> (o, lse)."""
+             need_lse=True, counter=None):
+    """bf16 prefill forward.  q: [B,H,Lq,d], k, v: [B,H,Lk,d] -> (o, lse).
+    ``counter`` (optional, a zeroed one-element int64 CUDA tensor) receives the
+    number of KV tiles visited."""
     _want(q, torch.bfloat16, 4, "q")
-    _want(k, torch.bfloat16, 4, "k")
-    _want(v, torch.bfloat16, 4, "v")
     B, H, Lq, d = q.shape
+    dev = q.device
+    _want(k, torch.bfloat16, 4, "k", device=dev)
     Lk = k.shape[2]
+    _want(k, torch.bfloat16, 4, "k", shape=(B, H, Lk, d))  # same batch, heads and head dim as q
+    _want(v, torch.bfloat16, 4, "v", shape=(B, H, Lk, d), device=dev)
+    _want_counter(counter, dev)
     if o is None:
         o = torch.empty_like(q)
+    _want(o, torch.bfloat16, 4, "o", shape=(B, H, Lq, d), device=dev)
     if lse is None and need_lse:
-        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _want(lse, torch.float32, 3, "lse", shape=(B, H, Lq), device=dev)
     scale = (1.0 / d ** 0.5) if scale is None else scale
-    _check(lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Lq, Lk, d, scale,
-                        int(bool(causal)), int(window_left), int(window_right), _stream()), "attn_fwd")
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Lq, Lk, d, scale, int(bool(causal)),
+            int(window_left), int(window_right))
+    if counter is None:
+        _check(lib.attn_fwd(*args, _stream()), "attn_fwd")
+    else:
+        _check(lib.attn_fwd_counted(*args, _ptr(counter), _stream()), "attn_fwd_counted")
     return o, lse
 
 
@@ -128,18 +160,7 @@ def attn_fwd_counted(q, k, v, counter, o=None, lse=None, scale=None, causal=Fals
                      window_right=-1):
     """attn_fwd that adds the number of KV tiles visited to ``counter``
     (a zeroed uint64/int64 CUDA tensor with one element)."""
-    _want(q, torch.bfloat16, 4, "q")
-    B, H, Lq, d = q.shape
-    Lk = k.shape[2]
-    if o is None:
-        o = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
-    scale = (1.0 / d ** 0.5) if scale is None else scale
-    _check(lib.attn_fwd_counted(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Lq, Lk, d, scale,
-                                int(bool(causal)), int(window_left), int(window_right), _ptr(counter),
-                                _stream()), "attn_fwd_counted")
-    return o, lse
+    return attn_fwd(q, k, v, o, lse, scale, causal, window_left, window_right, counter=counter)
 
 
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, o=None, lse=None, scale=None,
@@ -152,12 +173,20 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, o=None, l
     _want(cu_seqlens_q, torch.int32, 1, "cu_seqlens_q")
     _want(cu_seqlens_k, torch.int32, 1, "cu_seqlens_k")
     total_q, H, d = q.shape
+    dev = q.device
     total_k = k.shape[0]
     nseq = cu_seqlens_q.numel() - 1
+    _want(k, torch.bfloat16, 3, "k", shape=(total_k, H, d), device=dev)
+    _want(v, torch.bfloat16, 3, "v", shape=(total_k, H, d), device=dev)
+    _want(cu_seqlens_q, torch.int32, 1, "cu_seqlens_q", device=dev)
+    _want(cu_seqlens_k, torch.int32, 1, "cu_seqlens_k", shape=(nseq + 1,), device=dev)
+    _want_counter(counter, dev)
     if o is None:
         o = torch.empty_like(q)
+    _want(o, torch.bfloat16, 3, "o", shape=(total_q, H, d), device=dev)
     if lse is None:
-        lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+        lse = torch.empty((H, total_q), dtype=torch.float32, device=dev)
+    _want(lse, torch.float32, 2, "lse", shape=(H, total_q), device=dev)
     scale = (1.0 / d ** 0.5) if scale is None else scale
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), nseq, H, total_q,
             total_k, int(max_seqlen_q), d, scale, int(bool(causal)), int(window_left), int(window_right))
@@ -174,11 +203,16 @@ def attn_fwd_f32(q, k, v, o=None, lse=None, scale=None, causal=False, window_lef
     _want(k, torch.float32, 4, "k")
     _want(v, torch.float32, 4, "v")
     B, H, Lq, d = q.shape
+    dev = q.device
     Lk = k.shape[2]
+    _want(k, torch.float32, 4, "k", shape=(B, H, Lk, d), device=dev)
+    _want(v, torch.float32, 4, "v", shape=(B, H, Lk, d), device=dev)
     if o is None:
         o = torch.empty_like(q)
+    _want(o, torch.float32, 4, "o", shape=(B, H, Lq, d), device=dev)
     if lse is None:
-        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=dev)
+    _want(lse, torch.float32, 3, "lse", shape=(B, H, Lq), device=dev)
     scale = (1.0 / d ** 0.5) if scale is None else scale
     _check(lib.attn_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Lq, Lk, d, scale,
                             int(bool(causal)), int(window_left), int(window_right), _stream()), "attn_fwd_f32")
@@ -199,18 +233,26 @@ def attn_decode_splitkv(q, k_cache, v_cache, o=None, lse=None, seqlens_k=None, s
     _want(q, torch.bfloat16, 4, "q")
     _want(k_cache, torch.bfloat16, 4, "k_cache")
     _want(v_cache, torch.bfloat16, 4, "v_cache")
-    B, H, _, d = q.shape
+    B, H, Lq, d = q.shape
+    dev = q.device
+    if Lq != 1:
+        raise ValueError(f"q: decode takes one query per head, got Lq={Lq}")
     Lk = k_cache.shape[2]
+    _want(k_cache, torch.bfloat16, 4, "k_cache", shape=(B, H, Lk, d), device=dev)
+    _want(v_cache, torch.bfloat16, 4, "v_cache", shape=(B, H, Lk, d), device=dev)
     if o is None:
         o = torch.empty_like(q)
+    _want(o, torch.bfloat16, 4, "o", shape=(B, H, 1, d), device=dev)
     if lse is None:
-        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+        lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    _want(lse, torch.float32, 2, "lse", shape=(B, H), device=dev)
     if seqlens_k is not None:
-        _want(seqlens_k, torch.int32, 1, "seqlens_k")
+        _want(seqlens_k, torch.int32, 1, "seqlens_k", shape=(B,), device=dev)
     S = num_splits if num_splits > 0 else attn_decode_auto_splits(B, H, Lk, d)
     need = attn_decode_workspace_bytes(B, H, Lk, d, S)
     if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _want_workspace(workspace, dev)
     scale = (1.0 / d ** 0.5) if scale is None else scale
     _check(lib.attn_decode_splitkv(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
                                    _ptr(seqlens_k), B, H, Lk, d, scale, S, _ptr(workspace),
@@ -227,14 +269,21 @@ def attn_decode_splitkv_noalloc(q, k_cache, v_cache, o=None, lse=None, seqlens_k
     _want(q, torch.bfloat16, 4, "q")
     _want(k_cache, torch.bfloat16, 4, "k_cache")
     _want(v_cache, torch.bfloat16, 4, "v_cache")
-    B, H, _, d = q.shape
+    B, H, Lq, d = q.shape
+    dev = q.device
+    if Lq != 1:
+        raise ValueError(f"q: decode takes one query per head, got Lq={Lq}")
     Lk = k_cache.shape[2]
+    _want(k_cache, torch.bfloat16, 4, "k_cache", shape=(B, H, Lk, d), device=dev)
+    _want(v_cache, torch.bfloat16, 4, "v_cache", shape=(B, H, Lk, d), device=dev)
     if o is None:
         o = torch.empty_like(q)
+    _want(o, torch.bfloat16, 4, "o", shape=(B, H, 1, d), device=dev)
     if lse is None:
-        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+        lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    _want(lse, torch.float32, 2, "lse", shape=(B, H), device=dev)
     if seqlens_k is not None:
-        _want(seqlens_k, torch.int32, 1, "seqlens_k")
+        _want(seqlens_k, torch.int32, 1, "seqlens_k", shape=(B,), device=dev)
     scale = (1.0 / d ** 0.5) if scale is None else scale
     _check(lib.attn_decode_splitkv_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
                                            _ptr(seqlens_k), B, H, Lk, d, scale, int(num_splits), _stream()),
@@ -252,17 +301,27 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seqlens_k, o=None, lse=N
     _want(v_pages, torch.bfloat16, 4, "v_pages")
     _want(block_table, torch.int32, 2, "block_table")
     _want(seqlens_k, torch.int32, 1, "seqlens_k")
-    B, H, _, d = q.shape
+    B, H, Lq, d = q.shape
+    dev = q.device
+    if Lq != 1:
+        raise ValueError(f"q: decode takes one query per head, got Lq={Lq}")
     num_pages, page_size = k_pages.shape[0], k_pages.shape[1]
     max_pages = block_table.shape[1]
     Lk = max_pages * page_size
+    _want(k_pages, torch.bfloat16, 4, "k_pages", shape=(num_pages, page_size, H, d), device=dev)
+    _want(v_pages, torch.bfloat16, 4, "v_pages", shape=(num_pages, page_size, H, d), device=dev)
+    _want(block_table, torch.int32, 2, "block_table", shape=(B, max_pages), device=dev)
+    _want(seqlens_k, torch.int32, 1, "seqlens_k", shape=(B,), device=dev)
     if o is None:
         o = torch.empty_like(q)
+    _want(o, torch.bfloat16, 4, "o", shape=(B, H, 1, d), device=dev)
     if lse is None:
-        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+        lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    _want(lse, torch.float32, 2, "lse", shape=(B, H), device=dev)
     S = num_splits if num_splits > 0 else attn_decode_auto_splits(B, H, Lk, d)
     if workspace is None:
-        workspace = torch.empty(attn_decode_workspace_bytes(B, H, Lk, d, S), dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(attn_decode_workspace_bytes(B, H, Lk, d, S), dtype=torch.uint8, device=dev)
+    _want_workspace(workspace, dev)
     scale = (1.0 / d ** 0.5) if scale is None else scale
     _check(lib.attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), max_pages, page_size,
                                  num_pages, _ptr(o), _ptr(lse), _ptr(seqlens_k), B, H, d, scale, S, _ptr(workspace),
@@ -279,11 +338,14 @@ def attn_quantize_fp8(x, transpose=False, codes=None, descale=None):
     transposed; fp32 descale [B,H])."""
     _want(x, torch.bfloat16, 4, "x")
     B, H, L, d = x.shape
+    dev = x.device
+    shape = (B, H, d, attn_fp8_ld(L)) if transpose else (B, H, L, d)
     if codes is None:
-        shape = (B, H, d, attn_fp8_ld(L)) if transpose else (B, H, L, d)
-        codes = torch.empty(shape, dtype=torch.uint8, device=x.device)
+        codes = torch.empty(shape, dtype=torch.uint8, device=dev)
+    _want(codes, torch.uint8, 4, "codes", shape=shape, device=dev)
     if descale is None:
-        descale = torch.empty((B, H), dtype=torch.float32, device=x.device)
+        descale = torch.empty((B, H), dtype=torch.float32, device=dev)
+    _want(descale, torch.float32, 2, "descale", shape=(B, H), device=dev)
     _check(lib.attn_quantize_fp8(_ptr(x), _ptr(codes), _ptr(descale), B, H, L, d, int(bool(transpose)), _stream()),
            "attn_quantize_fp8")
     return codes, descale
@@ -298,13 +360,19 @@ def attn_fwd_fp8(q8, k8, vt8, q_descale, k_descale, v_descale, o=None, lse=None,
     for t, name in ((q_descale, "q_descale"), (k_descale, "k_descale"), (v_descale, "v_descale")):
         _want(t, torch.float32, 2, name)
     B, H, Lq, d = q8.shape
+    dev = q8.device
     Lk = k8.shape[2]
-    if tuple(vt8.shape) != (B, H, d, attn_fp8_ld(Lk)):
-        raise ValueError(f"vt8: expected shape {(B, H, d, attn_fp8_ld(Lk))}, got {tuple(vt8.shape)}")
+    _want(k8, torch.uint8, 4, "k8", shape=(B, H, Lk, d), device=dev)
+    _want(vt8, torch.uint8, 4, "vt8", shape=(B, H, d, attn_fp8_ld(Lk)), device=dev)
+    for t, name in ((q_descale, "q_descale"), (k_descale, "k_descale"), (v_descale, "v_descale")):
+        _want(t, torch.float32, 2, name, shape=(B, H), device=dev)
+    _want_counter(counter, dev)
     if o is None:
-        o = torch.empty((B, H, Lq, d), dtype=torch.bfloat16, device=q8.device)
+        o = torch.empty((B, H, Lq, d), dtype=torch.bfloat16, device=dev)
+    _want(o, torch.bfloat16, 4, "o", shape=(B, H, Lq, d), device=dev)
     if lse is None:
-        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q8.device)
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=dev)
+    _want(lse, torch.float32, 3, "lse", shape=(B, H, Lq), device=dev)
     scale = (1.0 / d ** 0.5) if scale is None else scale
     args = (_ptr(q8), _ptr(k8), _ptr(vt8), _ptr(q_descale), _ptr(k_descale), _ptr(v_descale), _ptr(o), _ptr(lse),
             B, H, Lq, Lk, d, scale, int(bool(causal)), int(window_left), int(window_right))
@@ -329,14 +397,21 @@ def attn_bwd(q, k, v, o, dout, lse, scale=None, causal=False, window_left=-1, wi
         _want(t, torch.bfloat16, 4, name)
     _want(lse, torch.float32, 3, "lse")
     B, H, Lq, d = q.shape
+    dev = q.device
     Lk = k.shape[2]
-    if o.shape != q.shape or dout.shape != q.shape or v.shape != k.shape or tuple(lse.shape) != (B, H, Lq):
-        raise ValueError("attn_bwd: inconsistent shapes")
+    for t, name, shp in ((k, "k", (B, H, Lk, d)), (v, "v", (B, H, Lk, d)), (o, "o", (B, H, Lq, d)),
+                         (dout, "dout", (B, H, Lq, d))):
+        _want(t, torch.bfloat16, 4, name, shape=shp, device=dev)
+    _want(lse, torch.float32, 3, "lse", shape=(B, H, Lq), device=dev)
+    _want_counter(counter, dev)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    for t, name, shp in ((dq, "dq", (B, H, Lq, d)), (dk, "dk", (B, H, Lk, d)), (dv, "dv", (B, H, Lk, d))):
+        _want(t, torch.bfloat16, 4, name, shape=shp, device=dev)
     if workspace is None:
-        workspace = torch.empty(attn_bwd_workspace_bytes(B, H, Lq, d), dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(attn_bwd_workspace_bytes(B, H, Lq, d), dtype=torch.uint8, device=dev)
+    _want_workspace(workspace, dev)
     scale = (1.0 / d ** 0.5) if scale is None else scale
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, H, Lq, Lk, d,
             scale, int(bool(causal)), int(window_left), int(window_right), _ptr(workspace),
