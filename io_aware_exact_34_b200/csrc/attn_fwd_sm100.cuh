@@ -43,6 +43,7 @@
 
 #include <cuda_bf16.h>
 #include <math_constants.h>
+#include <stddef.h>
 
 #include "dev_prims.cuh"
 #include "sched.cuh"
@@ -50,6 +51,31 @@
 namespace fattn {
 
 constexpr float kRescaleSlack = 8.0f;
+
+// Work order of packed variable-length batches.  The dense item space (pair
+// index descending, then sequence, then head) holds an item for every pair
+// index below max_seqlen_q / 256 in every sequence, so a batch of mixed
+// lengths interleaves empty items with full ones and the static round-robin
+// gives some CTAs far more work than others.  Each CTA therefore builds the
+// compacted order in shared memory: pair index descending (under causal
+// masking a pair's cost grows with its index), within one pair index only the
+// sequences that reach it, longest first and ties by sequence index, then the
+// heads.  With np_b = ceil(ceil(len_b / 128) / 2) pairs in sequence b,
+// gt[p] = #{b : np_b > p} sequences reach pair p; perm lists the sequences by
+// np_b descending, so those are perm[0, gt[p]); off[p] = H * sum_{p' > p}
+// gt[p'] is the first slot of pair p.  The table is a function of the offsets
+// alone, so every CTA builds the same one and the slots partition the items.
+constexpr int VL_MAX_SEQ = 2048;    // larger batches keep the dense order
+constexpr int VL_MAX_PAIRS = 1024;  // max_seqlen_q <= 262144
+struct VarlenOrder {
+    int np[VL_MAX_SEQ];
+    int perm[VL_MAX_SEQ];
+    int cursor[VL_MAX_PAIRS + 1];
+    int gt[VL_MAX_PAIRS + 1];
+    int off[VL_MAX_PAIRS + 1];
+    int n_items;
+};
+constexpr int VL_TABLE_BYTES = static_cast<int>(sizeof(VarlenOrder));
 
 template <int D, bool kFp8 = false>
 struct FwdTraits {
@@ -67,6 +93,9 @@ struct FwdTraits {
     static constexpr int NBAR = 2 + 2 * NSTAGE + 6 + 1;
     static constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NBAR * 8;
     static constexpr int SMEM_BYTES = SMEM_MISC_OFF + 16 + 1024;  // + alignment slack
+    // packed batches: the VarlenOrder table after the barriers
+    static constexpr int SMEM_VL_OFF = SMEM_MISC_OFF + 16;
+    static constexpr int SMEM_BYTES_VARLEN = SMEM_BYTES + VL_TABLE_BYTES;
     static constexpr int THREADS = 384;
     // Register split: warpgroup 0 (producer, MMA issuer) lowers to REGS_LOW,
     // the two softmax warpgroups raise to REGS_HIGH.  128*80 + 256*208 = 63488
@@ -82,7 +111,7 @@ struct FwdTraits {
     __host__ __device__ static constexpr uint32_t tm_o(int t) { return 256u + static_cast<uint32_t>(t) * D; }
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(!kFp8 || D == 128, "the FP8 path is built for d = 128");
-    static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert(SMEM_BYTES_VARLEN <= 232448, "shared memory");
 };
 
 struct FwdParams {
@@ -93,6 +122,7 @@ struct FwdParams {
     float scale_log2;  // scale * log2(e)
     int causal, window_left, window_right;
     int n_pairs, n_items;
+    int vl_order;  // packed batches: 1 = work items in the compacted VarlenOrder
     int inject_stall;  // test hook: CTA 0 never delivers its first K tile
     // packed variable-length batches (B = number of sequences): sequence b
     // owns tokens [cu_q[b], cu_q[b+1]) of Q/O and [cu_k[b], cu_k[b+1]) of K/V
@@ -148,6 +178,93 @@ __device__ __forceinline__ int snake_item(int round, int cta, int grid) {
     // Work items are ordered longest first; alternating the direction of
     // each round evens out the per-CTA total.
     return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
+}
+
+// Builds the VarlenOrder table.  Called by every thread of the CTA; on return
+// the table is visible to all of them.  Needs p.B <= VL_MAX_SEQ and
+// p.n_pairs <= VL_MAX_PAIRS (the host checks both).
+__device__ void varlen_order_build(const FwdParams& p, VarlenOrder* vo) {
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int NP = p.n_pairs;
+    for (int v = tid; v <= NP; v += nthr) vo->cursor[v] = 0;
+    __syncthreads();
+    // pairs per sequence, from the offsets clamped exactly as item_seq clamps them
+    auto clampi = [](int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); };
+    for (int b = tid; b < p.B; b += nthr) {
+        const int c0 = clampi(__ldg(p.cu_q + b), 0, p.total_q);
+        const int c1 = clampi(__ldg(p.cu_q + b + 1), c0, p.total_q);
+        const int nq = (c1 - c0 + 127) / 128;
+        const int np = (nq + 1) / 2 < NP ? (nq + 1) / 2 : NP;
+        vo->np[b] = np;
+        atomicAdd(&vo->cursor[np], 1);  // histogram of np
+    }
+    __syncthreads();
+    if (tid < 32) {
+        const int lane = tid;
+        const int n = NP + 1;
+        const int chunk = (n + 31) / 32;
+        const int a = lane * chunk < n ? lane * chunk : n;
+        const int e = a + chunk < n ? a + chunk : n;
+        // gt[v] = sum_{v' > v} hist[v']: suffix sums, one contiguous chunk of v per lane
+        int part = 0;
+        for (int v = a; v < e; ++v) part += vo->cursor[v];
+        int suf = part;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_down_sync(0xffffffffu, suf, o);
+            if (lane + o < 32) suf += x;
+        }
+        int run = suf - part;
+        for (int v = e - 1; v >= a; --v) {
+            const int h = vo->cursor[v];
+            vo->gt[v] = run;
+            vo->cursor[v] = run;  // first perm position of the sequences with np == v
+            run += h;
+        }
+        __syncwarp();
+        // off[v] = H * sum_{v' > v} gt[v']
+        part = 0;
+        for (int v = a; v < e; ++v) part += vo->gt[v];
+        suf = part;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_down_sync(0xffffffffu, suf, o);
+            if (lane + o < 32) suf += x;
+        }
+        run = suf - part;
+        for (int v = e - 1; v >= a; --v) {
+            vo->off[v] = p.H * run;
+            run += vo->gt[v];
+        }
+        if (lane == 0) vo->n_items = p.H * suf;
+        __syncwarp();
+        // stable scatter of the sequences into perm by np descending
+        for (int b0 = 0; b0 < p.B; b0 += 32) {
+            const int b = b0 + lane;
+            const int v = b < p.B ? vo->np[b] : -1;
+            const unsigned peers = __match_any_sync(0xffffffffu, v);
+            const int rank = __popc(peers & ((1u << lane) - 1u));
+            if (v > 0) vo->perm[vo->cursor[v] + rank] = b;
+            __syncwarp();
+            if (v > 0 && lane == 31 - __clz(peers)) vo->cursor[v] += __popc(peers);
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+}
+
+// Slot of the compacted order -> item index of the dense order, or -1 past
+// the last slot.  vo_s is the shared-window address of the table.
+__device__ __forceinline__ int varlen_slot_item(const FwdParams& p, uint32_t vo_s, int slot) {
+    if (slot >= lds_s32(vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, n_items)))) return -1;
+    const uint32_t off_s = vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, off));
+    int lo = 0, hi = p.n_pairs - 1;  // off[] is non-increasing and off[n_pairs - 1] = 0
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (lds_s32(off_s + 4u * mid) <= slot) hi = mid;
+        else lo = mid + 1;
+    }
+    const int j = slot - lds_s32(off_s + 4u * lo);
+    const int b = lds_s32(vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, perm)) + 4u * (j / p.H));
+    return (p.n_pairs - 1 - lo) * (p.B * p.H) + b * p.H + j % p.H;
 }
 
 template <bool kVarlen>
@@ -335,6 +452,9 @@ __global__ void __launch_bounds__(384, 1)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + T::SMEM_MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + T::SMEM_MISC_OFF + 4);
     int* status = &g_fattn_status;
+    const uint32_t vo_s = base + T::SMEM_VL_OFF;
+    const bool vl = kVarlen && p.vl_order;
+    if (vl) varlen_order_build(p, reinterpret_cast<VarlenOrder*>(gbase + T::SMEM_VL_OFF));
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -365,7 +485,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
-
+    
     if (warp < 4) {
       warpgroup_reg_lower<T::REGS_LOW>();
       if (warp == 0) {
@@ -374,8 +494,10 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t ring = 0, q_round = 0;
             bool ok = true;
             for (int round = 0; ok; ++round) {
-                const int item = snake_item(round, blockIdx.x, gridDim.x);
-                if (item >= p.n_items) break;
+                const int slot = snake_item(round, blockIdx.x, gridDim.x);
+                if (slot >= p.n_items) break;
+                const int item = vl ? varlen_slot_item(p, vo_s, slot) : slot;
+                if (item < 0) break;
                 const PairTiles ts = pair_tiles<kVarlen>(p, item);
                 if (ts.lo >= ts.hi) continue;
                 if (q_round > 0) {
@@ -434,8 +556,10 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t ring = 0, q_round = 0, p_cnt[2] = {0u, 0u};
             bool ok = true;
             for (int round = 0; ok; ++round) {
-                const int item = snake_item(round, blockIdx.x, gridDim.x);
-                if (item >= p.n_items) break;
+                const int slot = snake_item(round, blockIdx.x, gridDim.x);
+                if (slot >= p.n_items) break;
+                const int item = vl ? varlen_slot_item(p, vo_s, slot) : slot;
+                if (item < 0) break;
                 const PairTiles ts = pair_tiles<kVarlen>(p, item);
                 if (ts.lo >= ts.hi) continue;
                 ok = mbar_wait(q_full, q_round & 1u, abort_flag, status, -6);
@@ -524,8 +648,10 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t s_phase = 0, o_phase = 0;
         bool ok = true;
         for (int round = 0; ok; ++round) {
-            const int item = snake_item(round, blockIdx.x, gridDim.x);
-            if (item >= p.n_items) break;
+            const int slot = snake_item(round, blockIdx.x, gridDim.x);
+            if (slot >= p.n_items) break;
+            const int item = vl ? varlen_slot_item(p, vo_s, slot) : slot;
+                if (item < 0) break;
             const RowPlan rp = row_plan<D, kVarlen>(p, item, t, row);
             if (!rp.tile_exists) continue;
             float c_log2 = p.scale_log2, o_scale = 1.f;

@@ -89,8 +89,8 @@ int device_ready(DeviceInfo* out) {
             cudaError_t e = cudaSuccess;
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64>::SMEM_BYTES);
-            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128>::SMEM_BYTES);
-            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64>::SMEM_BYTES);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128>::SMEM_BYTES_VARLEN);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64>::SMEM_BYTES_VARLEN);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128, true>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_bwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdTraits<128>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_bwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdTraits<64>::SMEM_BYTES);
@@ -185,13 +185,18 @@ int encode_map_acc(CUtensorMap* map, float* base, int d, long long rows) {
     return r == CUDA_SUCCESS ? FATTN_OK : FATTN_ERR_CUDA;
 }
 
+template <int D, bool kVarlen>
+constexpr int fwd_smem_bytes() {
+    return kVarlen ? FwdTraits<D>::SMEM_BYTES_VARLEN : FwdTraits<D>::SMEM_BYTES;
+}
+
 template <bool kVarlen>
 int launch_prefill_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
                           int d, int grid, cudaStream_t s) {
     if (d == 128)
-        attn_fwd_sm100_kernel<128, kVarlen><<<grid, FwdTraits<128>::THREADS, FwdTraits<128>::SMEM_BYTES, s>>>(mq, mk, mv, p);
+        attn_fwd_sm100_kernel<128, kVarlen><<<grid, FwdTraits<128>::THREADS, fwd_smem_bytes<128, kVarlen>(), s>>>(mq, mk, mv, p);
     else
-        attn_fwd_sm100_kernel<64, kVarlen><<<grid, FwdTraits<64>::THREADS, FwdTraits<64>::SMEM_BYTES, s>>>(mq, mk, mv, p);
+        attn_fwd_sm100_kernel<64, kVarlen><<<grid, FwdTraits<64>::THREADS, fwd_smem_bytes<64, kVarlen>(), s>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? FATTN_OK : FATTN_ERR_CUDA;
 }
 
@@ -212,7 +217,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     if (encode_map(&mq, q, d, Lq, BH) != FATTN_OK || encode_map(&mk, k, d, Lk, BH) != FATTN_OK ||
         encode_map(&mv, v, d, Lk, BH) != FATTN_OK)
         return FATTN_ERR_CUDA;
-    FwdParams p;
+    FwdParams p{};
     p.o = o;
     p.lse = lse;
     p.visited = visited;
@@ -255,7 +260,7 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
     if (encode_map_packed(&mq, q, d, H, total_q) != FATTN_OK || encode_map_packed(&mk, k, d, H, total_k) != FATTN_OK ||
         encode_map_packed(&mv, v, d, H, total_k) != FATTN_OK)
         return FATTN_ERR_CUDA;
-    FwdParams p;
+    FwdParams p{};
     p.o = o;
     p.lse = lse;
     p.visited = visited;
@@ -274,6 +279,7 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
     p.cu_k = cu_k;
     p.total_q = total_q;
     p.total_k = total_k;
+    p.vl_order = (nseq <= VL_MAX_SEQ && n_pairs <= VL_MAX_PAIRS) ? 1 : 0;
     const int grid = static_cast<int>(n_items < di.num_sms ? n_items : di.num_sms);
     return launch_prefill_kernel<true>(mq, mk, mv, p, d, grid, static_cast<cudaStream_t>(stream));
 }
@@ -395,7 +401,7 @@ int launch_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float*
     if (encode_map_u8(&mq, q8, d, Lq, BH, d) != FATTN_OK || encode_map_u8(&mk, k8, d, Lk, BH, d) != FATTN_OK ||
         encode_map_u8(&mv, vt8, Lk, d, BH, fp8_ld(Lk)) != FATTN_OK)
         return FATTN_ERR_CUDA;
-    FwdParams p;
+    FwdParams p{};
     p.o = o;
     p.lse = lse;
     p.visited = visited;

@@ -22,11 +22,11 @@ def fl():
     return fattn
 
 
-def _check_varlen(fl, oracle, lens_q, lens_k, H, d, causal, wl, wr, seed):
+def _check_varlen(fl, oracle, lens_q, lens_k, H, d, causal, wl, wr, seed, max_q=None):
     q, k, v, cu_q, cu_k = synth.make_varlen_inputs(lens_q, lens_k, H, d, seed)
     counter = torch.zeros(1, dtype=torch.int64, device="cuda")
-    o, lse = fl.attn_fwd_varlen(q.cuda(), k.cuda(), v.cuda(), cu_q.cuda(), cu_k.cuda(), max(lens_q), causal=causal,
-                                window_left=wl, window_right=wr, counter=counter)
+    o, lse = fl.attn_fwd_varlen(q.cuda(), k.cuda(), v.cuda(), cu_q.cuda(), cu_k.cuda(), max_q or max(lens_q),
+                                causal=causal, window_left=wl, window_right=wr, counter=counter)
     torch.cuda.synchronize()
     o, lse = o.float().cpu().numpy(), lse.cpu().numpy()
     scale = d ** -0.5
@@ -70,3 +70,20 @@ def test_varlen_head_dim_64_and_empty_sequences(fl, oracle):
 def test_varlen_large_mix(fl, oracle):
     lens = synth.varlen_lengths(12, 256, 3000, seed=34)
     _check_varlen(fl, oracle, lens, lens, 4, 128, True, -1, -1, seed=35)
+
+
+def test_varlen_max_seqlen_above_every_length(fl, oracle):
+    # pair indices no sequence reaches: the compacted work order skips them
+    lens = [900, 130, 0, 2000, 256, 257]
+    _check_varlen(fl, oracle, lens, lens, 2, 128, True, -1, -1, seed=36, max_q=5000)
+
+
+@pytest.mark.parametrize("n_short", [2045, 2046])
+def test_varlen_many_sequences(fl, oracle, n_short):
+    # 2048 sequences take the compacted work order built in shared memory;
+    # 2049 exceed its table and take the dense order.  Both must give the
+    # same per-sequence results; a few long sequences give several pair indices.
+    g = np.random.default_rng(37)
+    lens = [int(x) for x in g.integers(0, 100, n_short)] + [1500, 777, 2100]
+    g.shuffle(lens)
+    _check_varlen(fl, oracle, lens, lens, 1, 64, True, -1, -1, seed=38)
