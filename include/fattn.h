@@ -125,6 +125,42 @@ int attn_fwd_varlen_counted(const void* q, const void* k, const void* v, void* o
                             unsigned long long* kv_tiles_visited, void* stream);
 
 /*
+ * attn_fwd_host -- attn_fwd on HOST buffers, with the host <-> device copies
+ * overlapped with the computation.  The B*H heads are independent problems
+ * (§5.3 parallelises over them), so the library takes them in chunks of G
+ * heads (about 32 MB of Q, K, V each, G chosen here): the copy of chunk c+1
+ * to the device, the kernel on chunk c and the copy of chunk c-1 back to the
+ * host run at the same time on three library-owned streams, through two
+ * chunk buffers in the caller's workspace.  Results are bit-identical to
+ * attn_fwd on the same data.
+ *
+ *   q, k, v   host, bf16 [B,H,Lq,d] / [B,H,Lk,d] / [B,H,Lk,d]; page-locked
+ *             (cudaHostAlloc / pinned) for the copies to overlap -- pageable
+ *             memory gives the same results with the copies serialised
+ *   o         host, bf16 [B,H,Lq,d] (written)
+ *   lse       host, fp32 [B,H,Lq] (written), or NULL to skip it
+ *   workspace device, 256-byte aligned, >= attn_fwd_host_workspace_bytes
+ *             bytes; caller-owned; not read or written after the call's work
+ *             on `stream` has completed
+ *   stream    the caller's stream: the work starts after what is already
+ *             queued on it, and work queued on it afterwards (for example a
+ *             cudaStreamSynchronize) sees o and lse complete
+ *   other arguments as attn_fwd
+ *
+ * Errors: as attn_fwd, plus FATTN_ERR_WORKSPACE for a null, misaligned or
+ * short workspace.  Calls from several host threads are serialised inside the
+ * library while they enqueue.
+ */
+int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                  int B, int H, int Lq, int Lk, int d, float scale,
+                  int causal, int window_left, int window_right,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Device workspace attn_fwd_host needs for these sizes (host only; 0 if the
+ * sizes are invalid). */
+size_t attn_fwd_host_workspace_bytes(int B, int H, int Lq, int Lk, int d);
+
+/*
  * attn_fwd_f32 -- the same operation on fp32 Q/K/V/O with fp32 arithmetic on
  * the CUDA cores (no tensor-core rounding), for exactness checks.  Arguments
  * as attn_fwd with fp32 tensors; d in {64, 128}; lse nullable.

@@ -438,11 +438,154 @@ int auto_splits(int B, int H, int Lk) {
 
 }  // namespace
 
+// ---------------------------------------------------------------- host-buffer prefill
+// Chunks of G heads: per head Q, K, V, O (bf16) and LSE (fp32), each array of
+// a chunk buffer starting on a 256-byte boundary; two chunk buffers.
+struct HostChunkPlan {
+    long long heads_per_chunk = 0;
+    size_t q_off = 0, k_off = 0, v_off = 0, o_off = 0, l_off = 0, chunk_bytes = 0;
+};
+
+size_t round_up256(size_t x) { return (x + 255) / 256 * 256; }
+
+bool host_chunk_plan(int B, int H, int Lq, int Lk, int d, HostChunkPlan* plan) {
+    if (B < 1 || H < 1 || Lq < 1 || Lk < 1 || (d != 64 && d != 128)) return false;
+    const long long BH = static_cast<long long>(B) * H;
+    const size_t qb = static_cast<size_t>(Lq) * d * 2, kb = static_cast<size_t>(Lk) * d * 2;
+    const size_t in_per_head = qb + 2 * kb;
+    long long g = static_cast<long long>((size_t{32} << 20) / in_per_head);
+    g = g < 1 ? 1 : (g > BH ? BH : g);
+    plan->heads_per_chunk = g;
+    const size_t G = static_cast<size_t>(g);
+    plan->q_off = 0;
+    plan->k_off = round_up256(G * qb);
+    plan->v_off = plan->k_off + round_up256(G * kb);
+    plan->o_off = plan->v_off + round_up256(G * kb);
+    plan->l_off = plan->o_off + round_up256(G * qb);
+    plan->chunk_bytes = plan->l_off + round_up256(G * static_cast<size_t>(Lq) * 4);
+    return true;
+}
+
+// Library-owned streams and events of one device for attn_fwd_host, created
+// on first use; g_host_mutex serialises the calls that enqueue on them.
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t h2d = nullptr, cmp = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, end = nullptr, in[2] = {}, done[2] = {}, freed[2] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_host_mutex;
+
+int host_pipe_ready(int dev, HostPipe** out) {
+    HostPipe& hp = g_pipe[dev];
+    if (!hp.ready) {
+        cudaError_t e = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking);
+        e = e != cudaSuccess ? e : cudaStreamCreateWithFlags(&hp.cmp, cudaStreamNonBlocking);
+        e = e != cudaSuccess ? e : cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking);
+        cudaEvent_t* evs[] = {&hp.start, &hp.end, &hp.in[0], &hp.in[1], &hp.done[0], &hp.done[1], &hp.freed[0], &hp.freed[1]};
+        for (cudaEvent_t* ev : evs) e = e != cudaSuccess ? e : cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return FATTN_ERR_CUDA;
+        }
+        hp.ready = true;
+    }
+    *out = &hp;
+    return FATTN_OK;
+}
+
+int fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq, int Lk, int d,
+             float scale, int causal, int wl, int wr, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!q || !k || !v || !o) return FATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return FATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FATTN_ERR_UNSUPPORTED;
+    HostChunkPlan plan;
+    if (!host_chunk_plan(B, H, Lq, Lk, d, &plan)) return FATTN_ERR_INVALID_ARG;
+    if (static_cast<long long>(B) * H > 0x7fffffffLL || Lq > 0x7fffff00 || Lk > 0x7fffff00) return FATTN_ERR_UNSUPPORTED;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < 2 * plan.chunk_bytes)
+        return FATTN_ERR_WORKSPACE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return FATTN_ERR_NO_DEVICE;
+    }
+    DeviceInfo di;
+    int st = device_ready(&di);
+    if (st != FATTN_OK) return st;
+    if (!di.fwd_regs_ok) return FATTN_ERR_UNSUPPORTED;
+
+    std::lock_guard<std::mutex> lock(g_host_mutex);
+    HostPipe* hp = nullptr;
+    st = host_pipe_ready(dev, &hp);
+    if (st != FATTN_OK) return st;
+    const cudaStream_t caller = static_cast<cudaStream_t>(stream);
+    const long long BH = static_cast<long long>(B) * H;
+    const size_t qb = static_cast<size_t>(Lq) * d * 2, kb = static_cast<size_t>(Lk) * d * 2, lb = static_cast<size_t>(Lq) * 4;
+    const long long G = plan.heads_per_chunk;
+    const long long n_chunks = (BH + G - 1) / G;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const uint8_t* qh = static_cast<const uint8_t*>(q);
+    const uint8_t* kh = static_cast<const uint8_t*>(k);
+    const uint8_t* vh = static_cast<const uint8_t*>(v);
+    uint8_t* oh = static_cast<uint8_t*>(o);
+    uint8_t* lh = reinterpret_cast<uint8_t*>(lse);
+
+    cudaError_t e = cudaEventRecord(hp->start, caller);
+    e = e != cudaSuccess ? e : cudaStreamWaitEvent(hp->h2d, hp->start, 0);
+    for (long long c = 0; c < n_chunks && e == cudaSuccess && st == FATTN_OK; ++c) {
+        const int b = static_cast<int>(c & 1);
+        const long long h0 = c * G;
+        const long long g = BH - h0 < G ? BH - h0 : G;
+        uint8_t* buf = ws + b * plan.chunk_bytes;
+        // chunk c reuses the buffer of chunk c - 2 once its copy back has finished
+        if (c >= 2) e = cudaStreamWaitEvent(hp->h2d, hp->freed[b], 0);
+        e = e != cudaSuccess ? e : cudaMemcpyAsync(buf + plan.q_off, qh + h0 * qb, g * qb, cudaMemcpyHostToDevice, hp->h2d);
+        e = e != cudaSuccess ? e : cudaMemcpyAsync(buf + plan.k_off, kh + h0 * kb, g * kb, cudaMemcpyHostToDevice, hp->h2d);
+        e = e != cudaSuccess ? e : cudaMemcpyAsync(buf + plan.v_off, vh + h0 * kb, g * kb, cudaMemcpyHostToDevice, hp->h2d);
+        e = e != cudaSuccess ? e : cudaEventRecord(hp->in[b], hp->h2d);
+        e = e != cudaSuccess ? e : cudaStreamWaitEvent(hp->cmp, hp->in[b], 0);
+        if (e != cudaSuccess) break;
+        float* lbuf = lse ? reinterpret_cast<float*>(buf + plan.l_off) : nullptr;
+        st = launch_fwd(buf + plan.q_off, buf + plan.k_off, buf + plan.v_off, buf + plan.o_off, lbuf, 1,
+                        static_cast<int>(g), Lq, Lk, d, scale, causal, wl, wr, nullptr, hp->cmp);
+        e = e != cudaSuccess ? e : cudaEventRecord(hp->done[b], hp->cmp);
+        e = e != cudaSuccess ? e : cudaStreamWaitEvent(hp->d2h, hp->done[b], 0);
+        e = e != cudaSuccess ? e : cudaMemcpyAsync(oh + h0 * qb, buf + plan.o_off, g * qb, cudaMemcpyDeviceToHost, hp->d2h);
+        if (lse) e = e != cudaSuccess ? e : cudaMemcpyAsync(lh + h0 * lb, lbuf, g * lb, cudaMemcpyDeviceToHost, hp->d2h);
+        e = e != cudaSuccess ? e : cudaEventRecord(hp->freed[b], hp->d2h);
+    }
+    // Whatever was queued (all of it, or a prefix after an error), the
+    // caller's stream waits for it: compute -> copy-back -> copy-in -> caller.
+    cudaError_t j = cudaEventRecord(hp->end, hp->cmp);
+    j = j != cudaSuccess ? j : cudaStreamWaitEvent(hp->d2h, hp->end, 0);
+    j = j != cudaSuccess ? j : cudaEventRecord(hp->end, hp->d2h);
+    j = j != cudaSuccess ? j : cudaStreamWaitEvent(hp->h2d, hp->end, 0);
+    j = j != cudaSuccess ? j : cudaEventRecord(hp->end, hp->h2d);
+    j = j != cudaSuccess ? j : cudaStreamWaitEvent(caller, hp->end, 0);
+    if (e != cudaSuccess || j != cudaSuccess) {
+        cudaGetLastError();
+        return FATTN_ERR_CUDA;
+    }
+    return st;
+}
+
 extern "C" {
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq, int Lk, int d,
              float scale, int causal, int window_left, int window_right, void* stream) {
     return launch_fwd(q, k, v, o, lse, B, H, Lq, Lk, d, scale, causal, window_left, window_right, nullptr, stream);
+}
+
+int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq, int Lk, int d,
+                  float scale, int causal, int window_left, int window_right, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+    return fwd_host(q, k, v, o, lse, B, H, Lq, Lk, d, scale, causal, window_left, window_right, workspace,
+                    workspace_bytes, stream);
+}
+
+size_t attn_fwd_host_workspace_bytes(int B, int H, int Lq, int Lk, int d) {
+    HostChunkPlan plan;
+    return host_chunk_plan(B, H, Lq, Lk, d, &plan) ? 2 * plan.chunk_bytes : 0;
 }
 
 int attn_fwd_counted(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq, int Lk,

@@ -23,6 +23,10 @@ _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_
 _llp = ctypes.POINTER(ctypes.c_longlong)
 lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp]
 lib.attn_fwd.restype = _i
+lib.attn_fwd_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp, ctypes.c_size_t, _vp]
+lib.attn_fwd_host.restype = _i
+lib.attn_fwd_host_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+lib.attn_fwd_host_workspace_bytes.restype = ctypes.c_size_t
 lib.attn_fwd_counted.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp, _vp]
 lib.attn_fwd_counted.restype = _i
 lib.attn_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp]
@@ -161,6 +165,52 @@ def attn_fwd_counted(q, k, v, counter, o=None, lse=None, scale=None, causal=Fals
     """attn_fwd that adds the number of KV tiles visited to ``counter``
     (a zeroed uint64/int64 CUDA tensor with one element)."""
     return attn_fwd(q, k, v, o, lse, scale, causal, window_left, window_right, counter=counter)
+
+
+def attn_fwd_host_workspace_bytes(B, H, Lq, Lk, d) -> int:
+    return lib.attn_fwd_host_workspace_bytes(B, H, Lq, Lk, d)
+
+
+def _want_host(t, dtype, ndim, name, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype or t.dim() != ndim or t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous {dtype} host tensor with {ndim} dims, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def attn_fwd_host(q, k, v, o=None, lse=None, scale=None, causal=False, window_left=-1, window_right=-1,
+                  need_lse=True, workspace=None):
+    """attn_fwd on host tensors (pin them for the copies to overlap the
+    kernels): q [B,H,Lq,d], k, v [B,H,Lk,d] bf16 on the CPU -> (o, lse) on the
+    CPU.  The device workspace is allocated here unless given (a uint8 CUDA
+    tensor of attn_fwd_host_workspace_bytes).  Returns once the results are in
+    o and lse (the current stream is synchronised)."""
+    _want_host(q, torch.bfloat16, 4, "q")
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2] if k.dim() == 4 else -1
+    _want_host(k, torch.bfloat16, 4, "k", shape=(B, H, Lk, d))
+    _want_host(v, torch.bfloat16, 4, "v", shape=(B, H, Lk, d))
+    if o is None:
+        o = torch.empty_like(q, pin_memory=True)
+    _want_host(o, torch.bfloat16, 4, "o", shape=(B, H, Lq, d))
+    if lse is None and need_lse:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, pin_memory=True)
+    if lse is not None:
+        _want_host(lse, torch.float32, 3, "lse", shape=(B, H, Lq))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    need = attn_fwd_host_workspace_bytes(B, H, Lq, Lk, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _want_workspace(workspace, dev)
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    _check(lib.attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Lq, Lk, d, scale,
+                             int(bool(causal)), int(window_left), int(window_right), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream()), "attn_fwd_host")
+    torch.cuda.current_stream().synchronize()
+    return o, lse
 
 
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, o=None, lse=None, scale=None,

@@ -240,3 +240,30 @@ def test_fp8_argument_checks(fl):
     if not torch.cuda.is_available():
         assert fwd() == fl.FATTN_ERR_NO_DEVICE
         assert q(FAKE, FAKE, FAKE, 1, 1, 10, 128, 1, None) == fl.FATTN_ERR_NO_DEVICE
+
+
+def test_host_prefill_argument_checks(fl):
+    lib = fl.lib
+    ws_need = fl.attn_fwd_host_workspace_bytes(2, 3, 300, 300, 128)
+    assert ws_need > 0
+    # invalid sizes give no workspace size
+    assert fl.attn_fwd_host_workspace_bytes(2, 3, 300, 300, 96) == 0
+    assert fl.attn_fwd_host_workspace_bytes(0, 3, 300, 300, 128) == 0
+    # two chunk buffers, each holding at least one head's Q, K, V, O and LSE
+    per_head = (300 * 128 * 2) * 4 + 300 * 4
+    assert ws_need >= 2 * per_head
+    # more heads never need less workspace; the chunk size is capped, so many heads need no more than a few
+    assert fl.attn_fwd_host_workspace_bytes(64, 16, 4096, 4096, 128) >= fl.attn_fwd_host_workspace_bytes(1, 1, 4096, 4096, 128)
+    assert fl.attn_fwd_host_workspace_bytes(64, 16, 4096, 4096, 128) == fl.attn_fwd_host_workspace_bytes(128, 16, 4096, 4096, 128)
+
+    def call(q=FAKE, k=FAKE, v=FAKE, o=FAKE, d=128, scale=0.1, ws=FAKE * 16, ws_bytes=None):
+        return lib.attn_fwd_host(q, k, v, o, None, 2, 3, 300, 300, d, scale, 1, -1, -1, ws,
+                                 ws_need if ws_bytes is None else ws_bytes, None)
+
+    assert call(q=None) == fl.FATTN_ERR_INVALID_ARG
+    assert call(o=None) == fl.FATTN_ERR_INVALID_ARG
+    assert call(scale=0.0) == fl.FATTN_ERR_INVALID_ARG
+    assert call(d=96) == fl.FATTN_ERR_UNSUPPORTED
+    assert call(ws=None) == fl.FATTN_ERR_WORKSPACE
+    assert call(ws=FAKE * 16 + 16) == fl.FATTN_ERR_WORKSPACE  # not 256-byte aligned
+    assert call(ws_bytes=ws_need - 1) == fl.FATTN_ERR_WORKSPACE
