@@ -123,6 +123,7 @@ struct FwdParams {
     int causal, window_left, window_right;
     int n_pairs, n_items;
     int vl_order;  // packed batches: 1 = work items in the compacted VarlenOrder
+    int o_vec32;   // O's base is 32-byte aligned: the epilogue writes 32-byte pieces of each row
     int inject_stall;  // test hook: CTA 0 never delivers its first K tile
     // packed variable-length batches (B = number of sequences): sequence b
     // owns tokens [cu_q[b], cu_q[b+1]) of Q/O and [cu_k[b], cu_k[b+1]) of K/V
@@ -754,9 +755,16 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         pk16[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l, __uint_as_float(orr[2 * e + 1]) * inv_l);
-                    uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+                    if (p.o_vec32) {
+                        stg256(orow + ch * 32, pk16[0], pk16[1], pk16[2], pk16[3], pk16[4], pk16[5], pk16[6], pk16[7]);
+                        stg256(orow + ch * 32 + 16, pk16[8], pk16[9], pk16[10], pk16[11], pk16[12], pk16[13], pk16[14],
+                               pk16[15]);
+                    } else {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk16[4 * v], pk16[4 * v + 1], pk16[4 * v + 2], pk16[4 * v + 3]);
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_uint4(pk16[4 * v], pk16[4 * v + 1], pk16[4 * v + 2], pk16[4 * v + 3]);
+                    }
                 }
             }
             if (rp.valid && p.lse)

@@ -109,6 +109,15 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                  : "memory");
 }
 
+// One 32-byte global store (the address must be 32-byte aligned): a full L2
+// sector per instruction instead of two half-sector 16-byte writes.
+__device__ __forceinline__ void stg256(void* p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4,
+                                       uint32_t a5, uint32_t a6, uint32_t a7) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a0), "r"(a1), "r"(a2),
+                 "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+                 : "memory");
+}
+
 // Makes this thread's generic-proxy shared-memory writes visible to later
 // async-proxy reads (tensor-core operands read through a descriptor).
 __device__ __forceinline__ void fence_proxy_async_smem() {

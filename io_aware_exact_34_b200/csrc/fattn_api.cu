@@ -219,6 +219,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
         return FATTN_ERR_CUDA;
     FwdParams p{};
     p.o = o;
+    p.o_vec32 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 ? 1 : 0;
     p.lse = lse;
     p.visited = visited;
     p.B = B;
@@ -262,6 +263,7 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
         return FATTN_ERR_CUDA;
     FwdParams p{};
     p.o = o;
+    p.o_vec32 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 ? 1 : 0;
     p.lse = lse;
     p.visited = visited;
     p.B = nseq;
@@ -403,6 +405,7 @@ int launch_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float*
         return FATTN_ERR_CUDA;
     FwdParams p{};
     p.o = o;
+    p.o_vec32 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 ? 1 : 0;
     p.lse = lse;
     p.visited = visited;
     p.B = B;

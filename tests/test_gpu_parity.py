@@ -250,3 +250,20 @@ def test_decode_full_size_sampled(fl, oracle):
         o_ref, lse_ref = oracle.attn(qs, ks, vs, w.scale)
         compare(o[b:b + 1, h:h + 1].float().cpu().numpy(), lse[b:b + 1, h:h + 1].cpu().numpy(),
                 o_ref, lse_ref[..., 0], BF16_O_MAXABS, BF16_O_RELL2, label=f"decode_32k {b},{h}")
+
+
+def test_output_base_16_not_32_byte_aligned(fl):
+    # the epilogue writes 32-byte pieces of each O row when O's base allows it
+    # and 16-byte pieces otherwise; both give the same bits
+    from io_aware_exact_34_b200 import synth
+    B, H, L, d = 1, 3, 300, 128
+    q, k, v = (t.cuda() for t in synth.random_qkv(B, H, L, L, d, "bf16", seed=21))
+    o_a, lse_a = fl.attn_fwd(q, k, v, causal=True)
+    buf = torch.empty(B * H * L * d + 16, dtype=torch.bfloat16, device="cuda")
+    base = buf.data_ptr() % 32
+    off = ((16 - base) % 32) // 2  # elements to a 16-byte but not 32-byte boundary
+    o_u = buf[off:off + B * H * L * d].view(B, H, L, d)
+    assert o_u.data_ptr() % 32 == 16
+    fl.attn_fwd(q, k, v, o=o_u, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o_a, o_u)
