@@ -77,7 +77,7 @@ struct VarlenOrder {
 };
 constexpr int VL_TABLE_BYTES = static_cast<int>(sizeof(VarlenOrder));
 
-template <int D, bool kFp8 = false>
+template <int D, bool kFp8 = false, bool kVarlen = false>
 struct FwdTraits {
     static constexpr int ELEM = kFp8 ? 1 : 2;      // bytes per element
     static constexpr int BQ = 128;                 // rows per Q tile (one per TMEM lane)
@@ -85,17 +85,24 @@ struct FwdTraits {
     static constexpr int CHUNK_BYTES = 128 * 128;  // 128 rows x 128 B: one 128-B swizzle column
     static constexpr int NCHUNK = D * ELEM / 128;
     static constexpr int TILE_BYTES = 128 * D * ELEM;
-    static constexpr int NSTAGE = TILE_BYTES == 32768 ? 4 : 8;  // K/V ring slots
-    static constexpr int KSTEPS_S = D * ELEM / 32;              // 32-byte K steps of S = Q K^T
+    static constexpr int KSTEPS_S = D * ELEM / 32;  // 32-byte K steps of S = Q K^T
+    // K/V ring slots: as many as fit beside the Q pair, the barriers (at most
+    // 512 bytes with the misc words), the packed-batch order table and the
+    // alignment slack.  K/V tiles come from DRAM whenever the batch's K and V
+    // outgrow L2, and the slots in flight hide that latency.
+    static constexpr int SMEM_LIMIT = 232448;
+    static constexpr int NSTAGE =
+        (SMEM_LIMIT - 2 * TILE_BYTES - 512 - (kVarlen ? VL_TABLE_BYTES : 0) - 1024) / TILE_BYTES;
     static constexpr int SMEM_Q_OFF = 0;
     static constexpr int SMEM_RING_OFF = 2 * TILE_BYTES;
     static constexpr int SMEM_BAR_OFF = SMEM_RING_OFF + NSTAGE * TILE_BYTES;
     static constexpr int NBAR = 2 + 2 * NSTAGE + 6 + 1;
     static constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NBAR * 8;
-    static constexpr int SMEM_BYTES = SMEM_MISC_OFF + 16 + 1024;  // + alignment slack
-    // packed batches: the VarlenOrder table after the barriers
+    // packed batches: the VarlenOrder table after the misc words
     static constexpr int SMEM_VL_OFF = SMEM_MISC_OFF + 16;
-    static constexpr int SMEM_BYTES_VARLEN = SMEM_BYTES + VL_TABLE_BYTES;
+    static constexpr int SMEM_BYTES = SMEM_VL_OFF + (kVarlen ? VL_TABLE_BYTES : 0) + 1024;  // + alignment slack
+    static_assert(NBAR * 8 + 16 <= 512, "barrier space");
+    static_assert(NSTAGE >= 4, "K/V ring");
     static constexpr int THREADS = 384;
     // Register split: warpgroup 0 (producer, MMA issuer) lowers to REGS_LOW,
     // the two softmax warpgroups raise to REGS_HIGH.  128*80 + 256*208 = 63488
@@ -111,7 +118,7 @@ struct FwdTraits {
     __host__ __device__ static constexpr uint32_t tm_o(int t) { return 256u + static_cast<uint32_t>(t) * D; }
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(!kFp8 || D == 128, "the FP8 path is built for d = 128");
-    static_assert(SMEM_BYTES_VARLEN <= 232448, "shared memory");
+    static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory");
 };
 
 struct FwdParams {
@@ -430,7 +437,7 @@ template <int D, bool kVarlen, bool kFp8 = false>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using T = FwdTraits<D, kFp8>;
+    using T = FwdTraits<D, kFp8, kVarlen>;
     static_assert(!(kFp8 && kVarlen), "the FP8 path takes dense batches");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);

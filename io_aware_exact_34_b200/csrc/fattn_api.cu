@@ -89,8 +89,8 @@ int device_ready(DeviceInfo* out) {
             cudaError_t e = cudaSuccess;
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64>::SMEM_BYTES);
-            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128>::SMEM_BYTES_VARLEN);
-            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64>::SMEM_BYTES_VARLEN);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128, false, true>::SMEM_BYTES);
+            e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<64, false, true>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_fwd_sm100_kernel<128, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdTraits<128, true>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_bwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdTraits<128>::SMEM_BYTES);
             e = e != cudaSuccess ? e : cudaFuncSetAttribute(attn_bwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdTraits<64>::SMEM_BYTES);
@@ -187,7 +187,7 @@ int encode_map_acc(CUtensorMap* map, float* base, int d, long long rows) {
 
 template <int D, bool kVarlen>
 constexpr int fwd_smem_bytes() {
-    return kVarlen ? FwdTraits<D>::SMEM_BYTES_VARLEN : FwdTraits<D>::SMEM_BYTES;
+    return FwdTraits<D, false, kVarlen>::SMEM_BYTES;
 }
 
 template <bool kVarlen>
