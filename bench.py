@@ -449,7 +449,7 @@ def run_ours(args, world, rank, local):
 
     # ---------------------------------------------------------------- other prefill workloads
     extra = {}
-    if not args.no_extra:
+    if not args.no_extra and not args.no_windows:
         for name in EXTRA:
             we = synth.WORKLOADS[name]
             f_e, c_e = prefill_flops(fattn, we)
@@ -487,6 +487,7 @@ def run_ours(args, world, rank, local):
         tf = f_v / (vms * 1e-3) / 1e12
         extra["varlen_causal_32seq"] = {"value": world * tf, "unit": "TFLOP/s", "ms_per_step": vms, "steps": vsteps,
                                         "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
+                                        "dram_bytes_per_launch": recorded_traffic(PREFILL_KERNEL, "varlen_causal_32seq"),
                                         "config": {"workload": "varlen_causal_32seq", "num_seqs": VARLEN_SEQS,
                                                    "seqlen_range": [VARLEN_MIN, VARLEN_MAX], "total_tokens": int(sum(lens)),
                                                    "H": VARLEN_H, "d": 128, "causal": True, "layout": "packed [total, H, d]"}}
@@ -523,6 +524,7 @@ def main():
     ap.add_argument("--no-clocks", action="store_true", help="no nvidia-smi sampling or soak (profiling runs)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-windows", action="store_true", help="skip the window and 64K lines (keeps varlen)")
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
