@@ -111,6 +111,15 @@ int attn_fwd_counted(const void* q, const void* k, const void* v, void* o, float
  * sequence's own lengths (bottom-right alignment when they differ).  Offsets
  * read from cu_seqlens are clamped into [0, total], so no access leaves the
  * tensors; a sequence with no query token writes nothing.
+ *
+ * Work order: batches of up to 2048 sequences (and max_seqlen_q <= 262144)
+ * are dealt item by item from a counter, longest sequences first, so that the
+ * CTAs stay busy to the end and the items in flight share few sequences' K/V
+ * in L2.  The counter is one of 64 library-owned counters, taken in turn and
+ * zeroed on `stream` before the kernel: up to 64 such launches may run at
+ * the same time on different streams (a captured graph keeps the counter of
+ * its capture, so one graph must not run concurrently with itself).  Larger
+ * batches use a static order.  Results do not depend on the order.
  */
 int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
                     const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs, int H,

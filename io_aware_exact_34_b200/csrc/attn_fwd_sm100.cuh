@@ -54,26 +54,28 @@ constexpr float kRescaleSlack = 8.0f;
 
 // Work order of packed variable-length batches.  The dense item space (pair
 // index descending, then sequence, then head) holds an item for every pair
-// index below max_seqlen_q / 256 in every sequence, so a batch of mixed
-// lengths interleaves empty items with full ones and the static round-robin
-// gives some CTAs far more work than others.  Each CTA therefore builds the
-// compacted order in shared memory: pair index descending (under causal
-// masking a pair's cost grows with its index), within one pair index only the
-// sequences that reach it, longest first and ties by sequence index, then the
-// heads.  With np_b = ceil(ceil(len_b / 128) / 2) pairs in sequence b,
-// gt[p] = #{b : np_b > p} sequences reach pair p; perm lists the sequences by
-// np_b descending, so those are perm[0, gt[p]); off[p] = H * sum_{p' > p}
-// gt[p'] is the first slot of pair p.  The table is a function of the offsets
-// alone, so every CTA builds the same one and the slots partition the items.
+// index below max_seqlen_q / 256 in every sequence; a batch of mixed lengths
+// makes most of them empty and the items' costs uneven.  Each CTA therefore
+// builds, in shared memory, a compacted order of the non-empty items:
+// sequences longest first (ties by sequence index), within a sequence its
+// pair indices descending (under causal masking a pair's cost grows with its
+// index), then the heads.  With np_b = ceil(ceil(len_b / 128) / 2) pairs in
+// sequence b, perm lists the sequences with np_b > 0 in that order and
+// seqoff[i] = H * sum_{i' < i} np_{perm[i']} is the first slot of perm[i].
+// The table is a function of the offsets alone, so every CTA builds the same
+// one.  The slots are dealt dynamically: the producer thread of a CTA takes
+// the next one from a per-launch counter when it starts an item, so CTAs that
+// drew short items take more of them, and the items in flight at any time
+// belong to few sequences, whose K and V stay in L2.
 constexpr int VL_MAX_SEQ = 2048;    // larger batches keep the dense order
 constexpr int VL_MAX_PAIRS = 1024;  // max_seqlen_q <= 262144
 struct VarlenOrder {
-    int np[VL_MAX_SEQ];
-    int perm[VL_MAX_SEQ];
-    int cursor[VL_MAX_PAIRS + 1];
-    int gt[VL_MAX_PAIRS + 1];
-    int off[VL_MAX_PAIRS + 1];
-    int n_items;
+    int np[VL_MAX_SEQ];           // pairs of sequence b
+    int perm[VL_MAX_SEQ];         // sequences by np descending
+    int seqoff[VL_MAX_SEQ + 1];   // first slot of perm[i]; seqoff[nne] = number of items
+    int cursor[VL_MAX_PAIRS + 1]; // histogram of np, then the bucket positions of the scatter
+    int nne;                      // sequences with at least one pair
+    int item_slot[2];             // the dealt items, handed from the producer to the other roles
 };
 constexpr int VL_TABLE_BYTES = static_cast<int>(sizeof(VarlenOrder));
 
@@ -96,7 +98,7 @@ struct FwdTraits {
     static constexpr int SMEM_Q_OFF = 0;
     static constexpr int SMEM_RING_OFF = 2 * TILE_BYTES;
     static constexpr int SMEM_BAR_OFF = SMEM_RING_OFF + NSTAGE * TILE_BYTES;
-    static constexpr int NBAR = 2 + 2 * NSTAGE + 6 + 1;
+    static constexpr int NBAR = 2 + 2 * NSTAGE + 6 + 1 + 4;
     static constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NBAR * 8;
     // packed batches: the VarlenOrder table after the misc words
     static constexpr int SMEM_VL_OFF = SMEM_MISC_OFF + 16;
@@ -129,7 +131,8 @@ struct FwdParams {
     float scale_log2;  // scale * log2(e)
     int causal, window_left, window_right;
     int n_pairs, n_items;
-    int vl_order;  // packed batches: 1 = work items in the compacted VarlenOrder
+    int vl_order;  // packed batches: 1 = work items in the compacted VarlenOrder, dealt by sched_ctr
+    unsigned int* sched_ctr;  // zeroed before the launch; the next slot to deal
     int o_vec32;   // O's base is 32-byte aligned: the epilogue writes 32-byte pieces of each row
     int inject_stall;  // test hook: CTA 0 never delivers its first K tile
     // packed variable-length batches (B = number of sequences): sequence b
@@ -213,7 +216,8 @@ __device__ void varlen_order_build(const FwdParams& p, VarlenOrder* vo) {
         const int chunk = (n + 31) / 32;
         const int a = lane * chunk < n ? lane * chunk : n;
         const int e = a + chunk < n ? a + chunk : n;
-        // gt[v] = sum_{v' > v} hist[v']: suffix sums, one contiguous chunk of v per lane
+        // first perm position of the sequences with np == v: the number with
+        // np > v, a suffix sum over the histogram, one contiguous chunk of v per lane
         int part = 0;
         for (int v = a; v < e; ++v) part += vo->cursor[v];
         int suf = part;
@@ -224,25 +228,10 @@ __device__ void varlen_order_build(const FwdParams& p, VarlenOrder* vo) {
         int run = suf - part;
         for (int v = e - 1; v >= a; --v) {
             const int h = vo->cursor[v];
-            vo->gt[v] = run;
-            vo->cursor[v] = run;  // first perm position of the sequences with np == v
+            vo->cursor[v] = run;
+            if (v == 0) vo->nne = run;  // sequences with np > 0
             run += h;
         }
-        __syncwarp();
-        // off[v] = H * sum_{v' > v} gt[v']
-        part = 0;
-        for (int v = a; v < e; ++v) part += vo->gt[v];
-        suf = part;
-        for (int o = 1; o < 32; o <<= 1) {
-            const int x = __shfl_down_sync(0xffffffffu, suf, o);
-            if (lane + o < 32) suf += x;
-        }
-        run = suf - part;
-        for (int v = e - 1; v >= a; --v) {
-            vo->off[v] = p.H * run;
-            run += vo->gt[v];
-        }
-        if (lane == 0) vo->n_items = p.H * suf;
         __syncwarp();
         // stable scatter of the sequences into perm by np descending
         for (int b0 = 0; b0 < p.B; b0 += 32) {
@@ -255,6 +244,21 @@ __device__ void varlen_order_build(const FwdParams& p, VarlenOrder* vo) {
             if (v > 0 && lane == 31 - __clz(peers)) vo->cursor[v] += __popc(peers);
             __syncwarp();
         }
+        // seqoff: exclusive prefix sums of H * np over perm, 32 sequences per step
+        const int nne = vo->nne;
+        int carry = 0;
+        for (int i0 = 0; i0 < nne; i0 += 32) {
+            const int i = i0 + lane;
+            const int x = i < nne ? vo->np[vo->perm[i]] : 0;
+            int inc = x;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += y;
+            }
+            if (i < nne) vo->seqoff[i] = p.H * (carry + inc - x);
+            carry += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) vo->seqoff[nne] = p.H * carry;
     }
     __syncthreads();
 }
@@ -262,17 +266,21 @@ __device__ void varlen_order_build(const FwdParams& p, VarlenOrder* vo) {
 // Slot of the compacted order -> item index of the dense order, or -1 past
 // the last slot.  vo_s is the shared-window address of the table.
 __device__ __forceinline__ int varlen_slot_item(const FwdParams& p, uint32_t vo_s, int slot) {
-    if (slot >= lds_s32(vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, n_items)))) return -1;
-    const uint32_t off_s = vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, off));
-    int lo = 0, hi = p.n_pairs - 1;  // off[] is non-increasing and off[n_pairs - 1] = 0
+    const int nne = lds_s32(vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, nne)));
+    const uint32_t so = vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, seqoff));
+    if (slot < 0 || slot >= lds_s32(so + 4u * nne)) return -1;
+    int lo = 0, hi = nne - 1;  // the last i with seqoff[i] <= slot (seqoff rises strictly)
     while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (lds_s32(off_s + 4u * mid) <= slot) hi = mid;
-        else lo = mid + 1;
+        const int mid = (lo + hi + 1) >> 1;
+        if (lds_s32(so + 4u * mid) <= slot) lo = mid;
+        else hi = mid - 1;
     }
-    const int j = slot - lds_s32(off_s + 4u * lo);
-    const int b = lds_s32(vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, perm)) + 4u * (j / p.H));
-    return (p.n_pairs - 1 - lo) * (p.B * p.H) + b * p.H + j % p.H;
+    const int s0 = lds_s32(so + 4u * lo);
+    const int npb = (lds_s32(so + 4u * (lo + 1)) - s0) / p.H;
+    const int local = slot - s0;
+    const int b = lds_s32(vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, perm)) + 4u * lo);
+    const int pair = npb - 1 - local / p.H;
+    return (p.n_pairs - 1 - pair) * (p.B * p.H) + b * p.H + local % p.H;
 }
 
 template <bool kVarlen>
@@ -457,6 +465,8 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t p_ready0 = s_full0 + 16;
     const uint32_t o_full0 = p_ready0 + 16;
     const uint32_t drain_bar = o_full0 + 16;
+    const uint32_t item_full0 = drain_bar + 8;    // [2]: the producer dealt an item (packed batches)
+    const uint32_t item_empty0 = item_full0 + 16;  // [2]: the MMA thread and the 8 softmax warps read it
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + T::SMEM_MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + T::SMEM_MISC_OFF + 4);
     int* status = &g_fattn_status;
@@ -477,6 +487,10 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(o_full0 + 8 * t, 1);
         }
         mbar_init(drain_bar, 1);
+        for (int e = 0; e < 2; ++e) {
+            mbar_init(item_full0 + 8 * e, 1);
+            mbar_init(item_empty0 + 8 * e, 9);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -502,9 +516,21 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t ring = 0, q_round = 0;
             bool ok = true;
             for (int round = 0; ok; ++round) {
-                const int slot = snake_item(round, blockIdx.x, gridDim.x);
-                if (slot >= p.n_items) break;
-                const int item = vl ? varlen_slot_item(p, vo_s, slot) : slot;
+                int item;
+                if (vl) {
+                    // deal: the next slot of the launch's counter, handed to the other roles
+                    item = varlen_slot_item(p, vo_s, static_cast<int>(atomicAdd(p.sched_ctr, 1u)));
+                    const int e = round & 1;
+                    if (round >= 2) {
+                        ok = mbar_wait(item_empty0 + 8 * e, ((round >> 1) - 1) & 1, abort_flag, status, -6);
+                        if (!ok) break;
+                    }
+                    sts_s32(vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, item_slot)) + 4u * e, item);
+                    mbar_arrive(item_full0 + 8 * e);
+                } else {
+                    const int slot = snake_item(round, blockIdx.x, gridDim.x);
+                    item = slot < p.n_items ? slot : -1;
+                }
                 if (item < 0) break;
                 const PairTiles ts = pair_tiles<kVarlen>(p, item);
                 if (ts.lo >= ts.hi) continue;
@@ -564,9 +590,17 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t ring = 0, q_round = 0, p_cnt[2] = {0u, 0u};
             bool ok = true;
             for (int round = 0; ok; ++round) {
-                const int slot = snake_item(round, blockIdx.x, gridDim.x);
-                if (slot >= p.n_items) break;
-                const int item = vl ? varlen_slot_item(p, vo_s, slot) : slot;
+                int item;
+                if (vl) {
+                    const int e = round & 1;
+                    ok = mbar_wait(item_full0 + 8 * e, (round >> 1) & 1, abort_flag, status, -6);
+                    if (!ok) break;
+                    item = lds_s32(vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, item_slot)) + 4u * e);
+                    mbar_arrive(item_empty0 + 8 * e);
+                } else {
+                    const int slot = snake_item(round, blockIdx.x, gridDim.x);
+                    item = slot < p.n_items ? slot : -1;
+                }
                 if (item < 0) break;
                 const PairTiles ts = pair_tiles<kVarlen>(p, item);
                 if (ts.lo >= ts.hi) continue;
@@ -656,10 +690,20 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t s_phase = 0, o_phase = 0;
         bool ok = true;
         for (int round = 0; ok; ++round) {
-            const int slot = snake_item(round, blockIdx.x, gridDim.x);
-            if (slot >= p.n_items) break;
-            const int item = vl ? varlen_slot_item(p, vo_s, slot) : slot;
-                if (item < 0) break;
+            int item;
+            if (vl) {
+                const int e = round & 1;
+                ok = mbar_wait(item_full0 + 8 * e, (round >> 1) & 1, abort_flag, status, -6);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                item = lds_s32(vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, item_slot)) + 4u * e);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(item_empty0 + 8 * e);
+            } else {
+                const int slot = snake_item(round, blockIdx.x, gridDim.x);
+                item = slot < p.n_items ? slot : -1;
+            }
+            if (item < 0) break;
             const RowPlan rp = row_plan<D, kVarlen>(p, item, t, row);
             if (!rp.tile_exists) continue;
             float c_log2 = p.scale_log2, o_scale = 1.f;

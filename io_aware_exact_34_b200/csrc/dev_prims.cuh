@@ -25,6 +25,10 @@ __device__ __forceinline__ int lds_s32(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ void sts_s32(uint32_t addr, int v) {
+    asm volatile("st.shared.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ unsigned long long global_timer_ns() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -63,6 +63,36 @@ std::atomic<int> g_inject_stall{0};
 __device__ __align__(256) float g_decode_noalloc_scratch[FATTN_DECODE_NOALLOC_SCRATCH_BYTES / sizeof(float)];
 void* g_noalloc_scratch_addr[kMaxDevices] = {};
 
+// Work counters of the packed prefill's dynamic deal: each launch takes the
+// next of kSchedSlots counters (a host ticket) and zeroes it on its stream, so
+// launches in flight at the same time use different counters as long as
+// fewer than kSchedSlots of them overlap.
+constexpr unsigned kSchedSlots = 64;
+__device__ unsigned int g_sched_ctr[kSchedSlots];
+unsigned int* g_sched_addr[kMaxDevices] = {};
+std::atomic<unsigned> g_sched_ticket{0};
+
+int sched_counter(unsigned int** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return FATTN_ERR_NO_DEVICE;
+    }
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (g_sched_addr[dev] == nullptr) {
+            void* addr = nullptr;
+            if (cudaGetSymbolAddress(&addr, g_sched_ctr) != cudaSuccess || addr == nullptr) {
+                cudaGetLastError();
+                return FATTN_ERR_CUDA;
+            }
+            g_sched_addr[dev] = static_cast<unsigned int*>(addr);
+        }
+    }
+    *out = g_sched_addr[dev] + (g_sched_ticket.fetch_add(1) % kSchedSlots);
+    return FATTN_OK;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Current device, checked to be sm_100 with the kernels' launch attributes set.
@@ -282,6 +312,14 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
     p.total_q = total_q;
     p.total_k = total_k;
     p.vl_order = (nseq <= VL_MAX_SEQ && n_pairs <= VL_MAX_PAIRS) ? 1 : 0;
+    if (p.vl_order) {
+        st = sched_counter(&p.sched_ctr);
+        if (st != FATTN_OK) return st;
+        if (cudaMemsetAsync(p.sched_ctr, 0, sizeof(unsigned int), static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+            cudaGetLastError();
+            return FATTN_ERR_CUDA;
+        }
+    }
     const int grid = static_cast<int>(n_items < di.num_sms ? n_items : di.num_sms);
     return launch_prefill_kernel<true>(mq, mk, mv, p, d, grid, static_cast<cudaStream_t>(stream));
 }
