@@ -33,7 +33,10 @@
  * is device memory owned by the caller, valid until the enqueued work is done.
  * Calls enqueue asynchronously on `stream` (a cudaStream_t, NULL = the legacy
  * default stream) and return once enqueued; the library allocates no device
- * memory.  Calls are thread-safe.
+ * memory.  Calls are thread-safe.  Library-owned state: a static decode
+ * scratch (attn_decode_splitkv_noalloc), 64 static work counters of the packed
+ * prefill (attn_fwd_varlen), and, from the first attn_fwd_host call on a
+ * device, three streams and eight events of that device.
  *
  * Errors.  Every entry point returns a fattn_status; nothing aborts or throws.
  * Argument checks run before any CUDA call, so a rejected call enqueues
