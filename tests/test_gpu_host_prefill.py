@@ -67,3 +67,32 @@ def test_host_prefill_rejects_device_tensors(fl):
     q = torch.zeros(1, 1, 8, 128, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(ValueError, match="host tensor"):
         fl.attn_fwd_host(q, q, q)
+
+
+def test_host_prefill_from_two_threads(fl):
+    # the library serialises the threads' enqueues on its own streams; each
+    # thread gets its own results
+    import threading
+    cases = [synth.random_qkv(1, 6, 700, 700, 128, "bf16", seed=s) for s in (11, 12)]
+    cases = [tuple(t.pin_memory() for t in c) for c in cases]
+    refs = [_device_reference(fl, *c, causal=True) for c in cases]
+    dev = torch.cuda.current_device()
+    results = [None, None]
+    errors = []
+
+    def work(n):
+        try:
+            torch.cuda.set_device(dev)
+            for _ in range(3):
+                results[n] = fl.attn_fwd_host(*cases[n], causal=True)
+                assert torch.equal(results[n][0], refs[n][0]) and torch.equal(results[n][1], refs[n][1])
+        except Exception as e:  # reported in the main thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=work, args=(n,)) for n in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not errors, errors
+    assert all(r is not None for r in results)

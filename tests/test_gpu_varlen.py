@@ -87,3 +87,28 @@ def test_varlen_many_sequences(fl, oracle, n_short):
     lens = [int(x) for x in g.integers(0, 100, n_short)] + [1500, 777, 2100]
     g.shuffle(lens)
     _check_varlen(fl, oracle, lens, lens, 1, 64, True, -1, -1, seed=38)
+
+
+def test_varlen_concurrent_streams(fl):
+    # launches in flight together on two streams draw different work counters
+    # and give the same bits as when run one at a time
+    lens_a = synth.varlen_lengths(9, 100, 1500, seed=41)
+    lens_b = synth.varlen_lengths(13, 50, 900, seed=42)
+    ins = []
+    for lens, seed in ((lens_a, 43), (lens_b, 44)):
+        q, k, v, cq, ck = synth.make_varlen_inputs(lens, lens, 4, 128, seed)
+        ins.append((q.cuda(), k.cuda(), v.cuda(), cq.cuda(), ck.cuda(), max(lens)))
+    refs = []
+    for q, k, v, cq, ck, m in ins:
+        o, lse = fl.attn_fwd_varlen(q, k, v, cq, ck, m, causal=True)
+        torch.cuda.synchronize()
+        refs.append((o.clone(), lse.clone()))
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    for it in range(6):
+        for (q, k, v, cq, ck, m), s in zip(ins, streams):
+            with torch.cuda.stream(s):
+                outs.append(fl.attn_fwd_varlen(q, k, v, cq, ck, m, causal=True))
+    torch.cuda.synchronize()
+    for n, (o, lse) in enumerate(outs):
+        assert torch.equal(o, refs[n % 2][0]) and torch.equal(lse, refs[n % 2][1]), f"launch {n}"
