@@ -424,7 +424,9 @@ def run_ours(args, world, rank, local):
     # ---------------------------------------------------------------- paged-KV decode
     decode_paged = None
     if not args.no_decode and not args.no_extra:
-        wd = synth.WORKLOADS[DECODE]
+        wd = dataclasses.replace(synth.WORKLOADS[DECODE], name=synth.WORKLOADS[DECODE].name + "_paged")
+        if args.decode_batch > 0:
+            wd = dataclasses.replace(wd, B=args.decode_batch, name=f"{wd.name}_b{args.decode_batch}")
         pq, kp, vp, table, seqlens = synth.make_paged_inputs(wd.B, wd.H, wd.Lk, wd.d, PAGE_SIZE,
                                                              seed=replica_seed(7, rank), device=dev)
         po = torch.empty_like(pq)
@@ -442,7 +444,12 @@ def run_ours(args, world, rank, local):
         gbs = pbytes / (pms * 1e-3) / 1e9
         decode_paged = {"metric": "decode HBM GB/s", "value": world * gbs, "unit": "GB/s", "ms_per_step": pms,
                         "steps": psteps, "frac_of_hbm_peak": gbs / peaks["hbm_gbs"],
-                        "config": {**wd.describe(), "workload": "decode_32k_paged", "page_size": PAGE_SIZE,
+                        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": gbs / peaks["hbm_gbs"],
+                                     "traffic": recorded_traffic("decode_split_kernel", wd.name),
+                                     "peak_source": f"{peak_src} copy bandwidth",
+                                     "kernels": ["decode_split_kernel", "decode_merge_kernel"]},
+                        "config": {**wd.describe(), "workload": wd.name, "page_size": PAGE_SIZE,
                                    "layout": "pages [num_pages, page_size, H, d], random block table"}}
         del pq, kp, vp, table, po, pws
         torch.cuda.empty_cache()
@@ -472,7 +479,7 @@ def run_ours(args, world, rank, local):
             torch.cuda.empty_cache()
 
     # ---------------------------------------------------------------- packed variable-length prefill
-    if not args.no_extra:
+    if not args.no_extra and not args.no_varlen:
         lens = synth.varlen_lengths(VARLEN_SEQS, VARLEN_MIN, VARLEN_MAX, seed=replica_seed(6, rank))
         vq, vk, vv, cuq, cuk = synth.make_varlen_inputs(lens, lens, VARLEN_H, 128, seed=replica_seed(6, rank), device=dev)
         vo = torch.empty_like(vq)
@@ -525,6 +532,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-windows", action="store_true", help="skip the window and 64K lines (keeps varlen)")
+    ap.add_argument("--no-varlen", action="store_true", help="skip the packed varlen line")
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
