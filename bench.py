@@ -2,15 +2,22 @@
 """Benchmark of libfattn on B200: one JSON line on stdout (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --sweep          # section 9.2 matrix, one JSON line per point
 
 A step is one pass of the prefill hot path (closed-form KV tile ranges, TMA
 Q/K/V tiles, tcgen05 S = Q K^T, masked exp2 online softmax, P V, O / l and
 LSE) over the causal 4 x 16 x 4096, d = 128 bf16 workload; ``value`` is its
 in-mask TFLOP/s (4 d FLOPs per allowed (q, k) pair per head) with inputs
-resident in HBM.  The same run times the backward with recomputation on that
-workload (``bwd``), the FP8 forward on it (``fp8``), the split-KV decode path (split kernel + LSE merge) on the
-64 x 32 x 32768 cache under ``decode`` in GB/s of K/V/q/o/lse traffic, and the
-sliding-window / long-causal prefill workloads under ``extra``.
+resident in HBM, the median of five timed regions of K steps (``repeats``).
+The same run reports: that step with L2 flushed before every launch
+(``cold_l2``); end to end on pinned host buffers (``e2e``); the backward with
+recomputation (``bwd``) and the FP8 forward (``fp8``) on that workload; the
+split-KV decode and its paged variant on the 64 x 32 x 32768 cache
+(``decode``, ``decode_paged``, GB/s); the d = 64 causal, sliding-window,
+long-causal and packed variable-length prefills (``extra``), each with its
+roofline; the fp64 oracle on the host cores (``cpu_baseline``: all cores,
+one core, sampled long workloads and decode slices with extrapolated full-run
+times).  ``summary``, the last key, repeats the headline figures compactly.
 
 Multi-GPU (torchrun, one rank per GPU): (batch, head) units are independent,
 so every rank runs its own full copy of the workload with no collective on the
@@ -33,7 +40,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "attention fwd TFLOP/s (in-mask FLOPs) & % bf16 tensor peak; decode HBM GB/s"
 HEADLINE = "causal_4k"
+HEADLINE_D64 = "causal_4k_d64"
+HEADLINE_REPEATS = 5
 DECODE = "decode_32k"
 EXTRA = ["window_bidir_32k", "window_causal_32k", "causal_64k_qscale"]
 VARLEN_SEQS, VARLEN_MIN, VARLEN_MAX, VARLEN_H = 32, 256, 4096, 16  # packed batch of causal requests
@@ -196,38 +206,168 @@ def timed(world, fn, steps, warmup):
     return max_over_ranks(world, start.elapsed_time(end) / steps)
 
 
+def timed_cold_l2(world, fn, steps, warmup, flush):
+    """Average device ms per step of fn when every step starts with a cold L2:
+    a write of `flush` (larger than L2) precedes each step outside the events
+    that bracket it.  Max over ranks."""
+    import torch
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(world, sum(a.elapsed_time(b) for a, b in evs) / steps)
+
+
 def prefill_flops(fl, w):
     c = fl.attn_count_blocks(w.Lq, w.Lk, w.causal, w.window_left, w.window_right, 128, 128)
     return 4.0 * w.d * c["pairs"] * w.B * w.H, c
 
 
-def cpu_baseline_sample(w, budget_s=12.0):
-    """The oracle, as it stands, on whole heads of the workload until about
-    `budget_s` seconds of work have run on all host cores."""
+def tensor_roofline(achieved, peaks, peak_src, kernel, traffic, scale=1.0, scale_note=""):
+    peak = peaks["bf16_tflops"] * scale
+    src = f"{peak_src} bf16 dense (burst)" + scale_note
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": traffic, "peak_source": src, "kernel": kernel}
+
+
+def r4(x):
+    """Four significant digits for the summary."""
+    if x is None:
+        return None
+    return float(f"{x:.4g}")
+
+
+# ---------------------------------------------------------------------- CPU baseline (the oracle)
+
+def allowed_keys(w, rows_i):
+    """Allowed keys of query rows rows_i (numpy int array) under w's mask:
+    accounting of the work a sampled row costs, not attention arithmetic."""
+    import numpy as np
+    i = np.asarray(rows_i, dtype=np.int64)
+    shift = w.Lk - w.Lq
+    lo = np.zeros_like(i)
+    hi = np.full_like(i, w.Lk - 1)
+    if w.window_left >= 0:
+        lo = np.maximum(lo, i + shift - w.window_left)
+    wr = w.window_right
+    if w.causal:
+        wr = 0 if wr < 0 else min(wr, 0)
+    if wr >= 0:
+        hi = np.minimum(hi, i + shift + wr)
+    return np.maximum(hi - lo + 1, 0)
+
+
+def cpu_sampled(w, full_heads, n_random, seed=7):
+    """The oracle on a stratified row sample of a long workload: every row of
+    `full_heads`, plus first / last rows, tile and window edges and `n_random`
+    random rows of every head.  Returns measured pairs/s and the full-run time
+    extrapolated from it."""
+    from io_aware_exact_34_b200 import synth
+    from oracle import oracle
+    q, k, v = synth.make_inputs(w)
+    rows = synth.sample_rows(w, n_random=n_random, seed=seed, full_heads=full_heads).numpy()
+    pairs = float(allowed_keys(w, rows[:, 2]).sum())
+    t0 = time.perf_counter()
+    oracle.attn_rows(q, k, v, rows, w.scale, w.causal, w.window_left, w.window_right)
+    dt = time.perf_counter() - t0
+    c = oracle.count_blocks(w.Lq, w.Lk, w.causal, w.window_left, w.window_right, 128, 128)
+    total_pairs = float(c["pairs"]) * w.B * w.H
+    pps = pairs / dt
+    return {"pairs_per_s": pps, "tflops": 4.0 * w.d * pps / 1e12, "rows": int(rows.shape[0]),
+            "full_heads": len(full_heads), "random_rows_per_head": n_random, "seconds": dt,
+            "extrapolated_full_run_s": total_pairs / pps, "extrapolated": True}
+
+
+def cpu_decode_slices(wd, n_slices, dev=None):
+    """The oracle on `n_slices` batch slices of the decode workload, one slice
+    at a time (32 heads x Lk keys each).  With `dev` the slices are cut from
+    the workload's own device-drawn cache and copied to the host one by one
+    (copy time excluded); otherwise each slice is drawn on the host with the
+    workload's distribution.  Returns K/V GB/s and the extrapolated full run."""
+    import torch
+    from io_aware_exact_34_b200 import synth
+    from oracle import oracle
+    kv_bytes = 2.0 * wd.H * wd.Lk * wd.d * 2  # bf16 K and V of one slice
+    dt = 0.0
+    if dev is not None:
+        q, k, v = synth.make_inputs(wd, device=dev)
+        for b in range(n_slices):
+            qs, ks, vs = (t[b:b + 1].cpu() for t in (q, k, v))
+            t0 = time.perf_counter()
+            oracle.attn(qs, ks, vs, wd.scale)
+            dt += time.perf_counter() - t0
+        del q, k, v
+        torch.cuda.empty_cache()
+    else:
+        for b in range(n_slices):
+            qs, ks, vs = synth.make_inputs(dataclasses.replace(wd, B=1), seed=wd.seed + 1000 + b)
+            t0 = time.perf_counter()
+            oracle.attn(qs, ks, vs, wd.scale)
+            dt += time.perf_counter() - t0
+    gbs = n_slices * kv_bytes / dt / 1e9
+    return {"gbs": gbs, "slices": n_slices, "of_slices": wd.B, "seconds": dt,
+            "extrapolated_full_run_s": wd.B * kv_bytes / (gbs * 1e9), "extrapolated": n_slices < wd.B,
+            "source": "device cache, copied per slice" if dev is not None else "host draw per slice"}
+
+
+def cpu_baseline(args, dev, budget_s=8.0):
+    """The oracle, as it stands, on the host cores: the headline workload on
+    whole heads for about `budget_s` seconds on all cores (the reported
+    baseline) and on one head with one thread (per-core figure); the long
+    prefill workloads on stratified row samples and the decode workload on
+    batch slices, each with its full-run time extrapolated.  --cpu-full takes
+    two full heads plus 4096 rows of every other head and every decode slice."""
     from io_aware_exact_34_b200 import synth
     from oracle import oracle
     oracle.build()
+    w = synth.WORKLOADS[HEADLINE]
     q, k, v = synth.make_inputs(w)
-    import torch
-    pairs_per_head = None
-    flops = 0.0
-    heads = 0
-    t0 = time.perf_counter()
+    cores = oracle.num_threads()
+    c = oracle.count_blocks(w.Lq, w.Lk, w.causal, w.window_left, w.window_right, 128, 128)
+    head_flops = 4.0 * w.d * c["pairs"]
+    heads, t0 = 0, time.perf_counter()
     for bh in range(w.B * w.H):
         b, h = divmod(bh, w.H)
         sl = (slice(b, b + 1), slice(h, h + 1))
         oracle.attn(q[sl], k[sl], v[sl], w.scale, w.causal, w.window_left, w.window_right)
-        if pairs_per_head is None:
-            c = oracle.count_blocks(w.Lq, w.Lk, w.causal, w.window_left, w.window_right, 128, 128)
-            pairs_per_head = c["pairs"]
-        flops += 4.0 * w.d * pairs_per_head
         heads += 1
         if time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
-    del torch
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{heads} of {w.B * w.H} (b,h) heads of {w.name}, every row, fp64, {dt:.1f} s"}
+    out = {"value": heads * head_flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+           "sample": f"{heads} of {w.B * w.H} (b,h) heads of {w.name}, every row, fp64, {dt:.1f} s on {cores} threads"}
+    # per-core figure: one whole head on one thread
+    oracle.set_num_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle.attn(q[:1, :1], k[:1, :1], v[:1, :1], w.scale, w.causal, w.window_left, w.window_right)
+        dt1 = time.perf_counter() - t0
+    finally:
+        oracle.set_num_threads(cores)
+    out["per_core"] = {"value": head_flops / dt1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                       "sample": f"head (0,0) of {w.name}, every row, one thread, {dt1:.1f} s"}
+    del q, k, v
+    cfgs = {}
+    for name in EXTRA:
+        we = synth.WORKLOADS[name]
+        if args.cpu_full:
+            fh, nr = [(0, 0), (0, we.H - 1)], 4096
+        else:
+            fh, nr = ([] if we.Lq > 32768 else [(0, 0)]), 256
+        cfgs[name] = cpu_sampled(we, fh, nr)
+    wd = synth.WORKLOADS[DECODE]
+    cfgs[DECODE] = cpu_decode_slices(wd, wd.B if args.cpu_full else 2, dev if args.cpu_full else None)
+    out["configs"] = cfgs
+    return out
 
 
 def run_reference(args, world, rank):
@@ -243,13 +383,13 @@ def run_reference(args, world, rank):
     g_rows = synth.sample_rows(w, n_random=0, seed=0, full_heads=[(w.B - 1, w.H - 1)]).numpy()
     g_rows = g_rows[g_rows[:, 0] == w.B - 1]
     g_rows = g_rows[g_rows[:, 1] == w.H - 1]
+
     # each step: 256 consecutive rows of the last head (every allowed key of each)
     def step(s):
         lo = (s * rows_per_step) % w.Lq
         rows = g_rows[lo:lo + rows_per_step]
         oracle.attn_rows(q, k, v, rows, w.scale, w.causal, w.window_left, w.window_right)
-        i = rows[:, 2]
-        return float(4.0 * w.d * (i + 1).sum())  # causal: row i has i + 1 keys
+        return float(4.0 * w.d * allowed_keys(w, rows[:, 2]).sum())
     for s in range(args.warmup):
         step(s)
     t0 = time.perf_counter()
@@ -258,7 +398,7 @@ def run_reference(args, world, rank):
         flops += step(args.warmup + s)
     dt = time.perf_counter() - t0
     value = flops / dt / 1e12
-    line = {"metric": "attention fwd TFLOP/s (in-mask FLOPs)", "value": value, "unit": "TFLOP/s",
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s",
             "impl": "reference", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -269,11 +409,88 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------- GPU lines
+
+def prefill_line(world, rank, dev, fl, peaks, peak_src, name, steps, warmup=3):
+    """One dense prefill workload: TFLOP/s on in-mask FLOPs, roofline, tiles."""
+    import torch
+    from io_aware_exact_34_b200 import synth
+    we = synth.WORKLOADS[name]
+    f_e, c_e = prefill_flops(fl, we)
+    eq, ek, ev = synth.make_inputs(we, device=dev, seed=replica_seed(we.seed, rank))
+    eo = torch.empty_like(eq)
+    el = torch.empty((we.B, we.H, we.Lq), dtype=torch.float32, device=dev)
+
+    def estep():
+        fl.attn_fwd(eq, ek, ev, o=eo, lse=el, scale=we.scale, causal=we.causal,
+                    window_left=we.window_left, window_right=we.window_right)
+
+    ems = timed(world, estep, steps, warmup)
+    tf = f_e / (ems * 1e-3) / 1e12
+    line = {"value": world * tf, "unit": "TFLOP/s", "ms_per_step": ems, "steps": steps,
+            "roofline": tensor_roofline(tf, peaks, peak_src, PREFILL_KERNEL, recorded_traffic(PREFILL_KERNEL, name)),
+            "kv_tiles_visited_per_head": c_e["visited"], "kv_tiles_total_per_head": c_e["total"],
+            "config": we.describe(), "gpu_launches": steps}
+    del eq, ek, ev, eo, el
+    torch.cuda.empty_cache()
+    return line
+
+
+def run_sweep(args, world, rank, dev, fl, peaks, peak_src):
+    """The experiment matrix of the sliding-window prefill page, section 9.2:
+    sequence length x window x batch, the tiled kernel with full attention
+    against the same kernel with the bidirectional window |i - j| <= w (out-of-
+    band tiles skipped).  One JSON line per point: times, TFLOP/s, tiles
+    visited, peak device memory, and the measured speedup beside the page's
+    n / (2w) estimate and the exact in-band pair ratio."""
+    import torch
+    from io_aware_exact_34_b200 import synth
+    H, d = args.sweep_heads, 128
+    for L in (4096, 8192, 16384, 32768):
+        for B in (1, 2, 4, 8):
+            torch.cuda.reset_peak_memory_stats()
+            wf = synth.Workload(f"sweep_full_{B}x{L}", "prefill", B, H, L, L, d, "bf16", seed=9)
+            q, k, v = synth.make_inputs(wf, device=dev, seed=replica_seed(9, rank))
+            o = torch.empty_like(q)
+            lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+            res = {}
+            for wsz in (None, 2048, 1024, 512):
+                wl = -1 if wsz is None else wsz
+
+                def st():
+                    fl.attn_fwd(q, k, v, o=o, lse=lse, window_left=wl, window_right=wl)
+
+                steps = 3 if L * L * B >= 8 * 16384 * 16384 else 10
+                ms = timed(world, st, steps, 3)
+                c = fl.attn_count_blocks(L, L, False, wl, wl, 128, 128)
+                fl_ = 4.0 * d * c["pairs"] * B * H
+                res[wsz] = (ms, fl_, c)
+            ms_full = res[None][0]
+            for wsz in (None, 2048, 1024, 512):
+                ms, fl_, c = res[wsz]
+                tf = fl_ / (ms * 1e-3) / 1e12
+                point = {"sweep": "p2_9.2", "seq": L, "batch": B, "heads": H, "d": d,
+                         "window": "full" if wsz is None else wsz, "ms": ms, "tflops": tf,
+                         "frac": tf / peaks["bf16_tflops"], "tiles_visited_per_head": c["visited"],
+                         "tiles_total_per_head": c["total"],
+                         "peak_mem_gb": torch.cuda.max_memory_allocated() / 1e9}
+                if wsz is not None:
+                    point.update(speedup_vs_full=ms_full / ms, page_estimate_n_over_2w=L / (2.0 * wsz),
+                                 exact_pair_ratio=res[None][2]["pairs"] / c["pairs"])
+                if rank == 0:
+                    print(json.dumps(point), flush=True)
+            del q, k, v, o, lse
+            torch.cuda.empty_cache()
+
+
 def run_ours(args, world, rank, local):
     import torch
     from io_aware_exact_34_b200 import fattn, synth
     peaks, peak_src = load_peaks()
     dev = torch.device("cuda", torch.cuda.current_device())
+    if args.sweep:
+        run_sweep(args, world, rank, dev, fattn, peaks, peak_src)
+        return
 
     # ---------------------------------------------------------------- headline prefill
     w = synth.WORKLOADS[HEADLINE]
@@ -286,27 +503,41 @@ def run_ours(args, world, rank, local):
         fattn.attn_fwd(q, k, v, o=o, lse=lse, scale=w.scale, causal=w.causal,
                        window_left=w.window_left, window_right=w.window_right)
 
-    if args.no_headline:
-        ms, clocks, value, roofline = float("nan"), None, None, None
-    elif args.no_clocks:
-        ms = timed(world, step, args.steps, args.warmup)
-        clocks = None
-    else:
-        with ClockSampler(local) as clk:
-            ms = timed(world, step, args.steps, args.warmup)
-            # keep the same work running for about a second so the sampler sees it
-            t_end = time.perf_counter() + 1.0
-            while time.perf_counter() < t_end:
-                for _ in range(20):
-                    step()
-                torch.cuda.synchronize()
-        clocks = clk.summary()
+    ms, clocks, value, roofline, repeats, cold = float("nan"), None, None, None, None, None
     if not args.no_headline:
+        def headline_regions():
+            # the K-step region timed HEADLINE_REPEATS times; the median is the line's time
+            out = [timed(world, step, args.steps, args.warmup)]
+            for _ in range(HEADLINE_REPEATS - 1):
+                out.append(timed(world, step, args.steps, 3))
+            return out
+
+        if args.no_clocks:
+            reps = headline_regions()
+        else:
+            with ClockSampler(local) as clk:
+                reps = headline_regions()
+                # keep the same work running for about a second so the sampler sees it
+                t_end = time.perf_counter() + 1.0
+                while time.perf_counter() < t_end:
+                    for _ in range(20):
+                        step()
+                    torch.cuda.synchronize()
+            clocks = clk.summary()
+        ms = statistics.median(reps)
         value = world * flops / (ms * 1e-3) / 1e12
         achieved = flops / (ms * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": achieved / peaks["bf16_tflops"], "traffic": recorded_traffic(PREFILL_KERNEL, w.name),
-                    "peak_source": f"{peak_src} bf16 dense (burst)", "kernel": PREFILL_KERNEL}
+        roofline = tensor_roofline(achieved, peaks, peak_src, PREFILL_KERNEL, recorded_traffic(PREFILL_KERNEL, w.name))
+        repeats = {"n": len(reps), "steps_each": args.steps, "ms_per_step": reps, "median": ms,
+                   "min": min(reps), "max": max(reps), "spread_pct": 100.0 * (max(reps) - min(reps)) / ms}
+        # the same step with L2 flushed (a 256 MB write) before each launch
+        flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+        cms = timed_cold_l2(world, step, args.steps, 3, flush)
+        del flush
+        ctf = flops / (cms * 1e-3) / 1e12
+        cold = {"value": world * ctf, "unit": "TFLOP/s", "ms_per_step": cms, "steps": args.steps,
+                "l2": "256 MB written before every step, outside its events",
+                "roofline": tensor_roofline(ctf, peaks, peak_src, PREFILL_KERNEL, None)}
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
@@ -345,13 +576,11 @@ def run_ours(args, world, rank, local):
         bms = timed(world, bstep, bsteps, 3)
         bflops = 2.5 * flops  # five products per allowed pair instead of two
         tf = bflops / (bms * 1e-3) / 1e12
+        rl = tensor_roofline(tf, peaks, peak_src, "attn_bwd_sm100_kernel",
+                             recorded_traffic("attn_bwd_sm100_kernel", w.name))
+        rl["kernels"] = ["bwd_prep_kernel", "attn_bwd_sm100_kernel", "bwd_dq_kernel"]
         bwd = {"metric": "attention bwd TFLOP/s (in-mask FLOPs: 10 d per allowed pair)", "value": world * tf,
-               "unit": "TFLOP/s", "ms_per_step": bms, "steps": bsteps,
-               "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                            "frac": tf / peaks["bf16_tflops"],
-                            "traffic": recorded_traffic("attn_bwd_sm100_kernel", w.name),
-                            "peak_source": f"{peak_src} bf16 dense (burst)",
-                            "kernels": ["bwd_prep_kernel", "attn_bwd_sm100_kernel", "bwd_dq_kernel"]},
+               "unit": "TFLOP/s", "ms_per_step": bms, "steps": bsteps, "roofline": rl,
                "config": {**w.describe(), "pass": "backward with recomputation from LSE"},
                "gpu_launches": 3 * bsteps}
         del dout, gq, gk, gv, gws
@@ -376,20 +605,21 @@ def run_ours(args, world, rank, local):
 
         fsteps = max(3, min(args.steps, 20))
         fms = timed(world, fstep, fsteps, 3)
-        qms = timed(world, qstep, 3, 3)
+        qms = timed(world, qstep, 5, 3)
         tf = flops / (fms * 1e-3) / 1e12
-        fp8_peak = 2.0 * peaks["bf16_tflops"]  # nominal dense fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s)
+        # nominal dense fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s) times the measured bf16 peak
+        rl = tensor_roofline(tf, peaks, peak_src, PREFILL_KERNEL + "<128, false, true>",
+                             recorded_traffic("attn_fwd_fp8", w.name), 2.0, " x 2 (nominal fp8/bf16 ratio)")
         fp8 = {"metric": "attention fwd TFLOP/s (in-mask FLOPs), e4m3 Q/K/V/P", "value": world * tf,
-               "unit": "TFLOP/s", "ms_per_step": fms, "steps": fsteps,
-               "roofline": {"bound": "tensor", "achieved": tf, "peak": fp8_peak, "unit": "TFLOP/s",
-                            "frac": tf / fp8_peak, "traffic": recorded_traffic("attn_fwd_fp8", w.name),
-                            "peak_source": f"{peak_src} bf16 dense (burst) x 2 (nominal fp8/bf16 ratio)",
-                            "kernel": PREFILL_KERNEL + "<128, false, true>"},
+               "unit": "TFLOP/s", "ms_per_step": fms, "steps": fsteps, "roofline": rl,
                "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
-               "quantize_ms_per_step": qms, "config": {**w.describe(), "dtype": "e4m3 (P e4m3, O bf16)"},
-               "gpu_launches": fsteps}
+               "quantize_ms_per_step": qms,
+               "quantize_then_attend_tflops": world * flops / ((fms + qms) * 1e-3) / 1e12,
+               "config": {**w.describe(), "dtype": "e4m3 (P e4m3, O bf16)"}, "gpu_launches": fsteps}
         del q8, k8, vt8, qs, ks, vs, o8
         torch.cuda.empty_cache()
+    del q, k, v, o, lse
+    torch.cuda.empty_cache()
 
     # ---------------------------------------------------------------- decode
     decode = None
@@ -443,40 +673,26 @@ def run_ours(args, world, rank, local):
         pbytes = (kp.numel() + vp.numel() + pq.numel() + po.numel()) * 2 + pl.numel() * 4 + table.numel() * 4
         gbs = pbytes / (pms * 1e-3) / 1e9
         decode_paged = {"metric": "decode HBM GB/s", "value": world * gbs, "unit": "GB/s", "ms_per_step": pms,
-                        "steps": psteps, "frac_of_hbm_peak": gbs / peaks["hbm_gbs"],
+                        "steps": psteps,
                         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                      "frac": gbs / peaks["hbm_gbs"],
                                      "traffic": recorded_traffic("decode_split_kernel", wd.name),
                                      "peak_source": f"{peak_src} copy bandwidth",
                                      "kernels": ["decode_split_kernel", "decode_merge_kernel"]},
                         "config": {**wd.describe(), "workload": wd.name, "page_size": PAGE_SIZE,
-                                   "layout": "pages [num_pages, page_size, H, d], random block table"}}
+                                   "layout": "pages [num_pages, page_size, H, d], random block table"},
+                        "gpu_launches": 2 * psteps}
         del pq, kp, vp, table, po, pws
         torch.cuda.empty_cache()
 
     # ---------------------------------------------------------------- other prefill workloads
     extra = {}
+    if not args.no_extra:
+        extra[HEADLINE_D64] = prefill_line(world, rank, dev, fattn, peaks, peak_src, HEADLINE_D64,
+                                           max(3, min(args.steps, 20)))
     if not args.no_extra and not args.no_windows:
         for name in EXTRA:
-            we = synth.WORKLOADS[name]
-            f_e, c_e = prefill_flops(fattn, we)
-            eq, ek, ev = synth.make_inputs(we, device=dev, seed=replica_seed(we.seed, rank))
-            eo = torch.empty_like(eq)
-            el = torch.empty((we.B, we.H, we.Lq), dtype=torch.float32, device=dev)
-
-            def estep():
-                fattn.attn_fwd(eq, ek, ev, o=eo, lse=el, scale=we.scale, causal=we.causal,
-                               window_left=we.window_left, window_right=we.window_right)
-
-            esteps = max(3, min(args.steps, 10))
-            ems = timed(world, estep, esteps, 2)
-            tf = f_e / (ems * 1e-3) / 1e12
-            extra[name] = {"value": world * tf, "unit": "TFLOP/s", "ms_per_step": ems, "steps": esteps,
-                           "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
-                           "kv_tiles_visited_per_head": c_e["visited"], "kv_tiles_total_per_head": c_e["total"],
-                           "config": we.describe()}
-            del eq, ek, ev, eo, el
-            torch.cuda.empty_cache()
+            extra[name] = prefill_line(world, rank, dev, fattn, peaks, peak_src, name, max(3, min(args.steps, 10)))
 
     # ---------------------------------------------------------------- packed variable-length prefill
     if not args.no_extra and not args.no_varlen:
@@ -490,33 +706,53 @@ def run_ours(args, world, rank, local):
             fattn.attn_fwd_varlen(vq, vk, vv, cuq, cuk, max(lens), o=vo, lse=vl, causal=True)
 
         vsteps = max(3, min(args.steps, 10))
-        vms = timed(world, vstep, vsteps, 2)
+        vms = timed(world, vstep, vsteps, 3)
         tf = f_v / (vms * 1e-3) / 1e12
-        extra["varlen_causal_32seq"] = {"value": world * tf, "unit": "TFLOP/s", "ms_per_step": vms, "steps": vsteps,
-                                        "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
-                                        "dram_bytes_per_launch": recorded_traffic(PREFILL_KERNEL, "varlen_causal_32seq"),
-                                        "config": {"workload": "varlen_causal_32seq", "num_seqs": VARLEN_SEQS,
-                                                   "seqlen_range": [VARLEN_MIN, VARLEN_MAX], "total_tokens": int(sum(lens)),
-                                                   "H": VARLEN_H, "d": 128, "causal": True, "layout": "packed [total, H, d]"}}
+        extra["varlen_causal_32seq"] = {
+            "value": world * tf, "unit": "TFLOP/s", "ms_per_step": vms, "steps": vsteps,
+            "roofline": tensor_roofline(tf, peaks, peak_src, PREFILL_KERNEL + "<128, true, false>",
+                                        recorded_traffic(PREFILL_KERNEL, "varlen_causal_32seq")),
+            "config": {"workload": "varlen_causal_32seq", "num_seqs": VARLEN_SEQS,
+                       "seqlen_range": [VARLEN_MIN, VARLEN_MAX], "total_tokens": int(sum(lens)),
+                       "H": VARLEN_H, "d": 128, "causal": True, "layout": "packed [total, H, d]"},
+            "gpu_launches": vsteps}
         del vq, vk, vv, vo, vl
         torch.cuda.empty_cache()
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_sample(w)
+        cpu = cpu_baseline(args, dev)
 
     if rank == 0:
-        line = {"metric": "attention fwd TFLOP/s (in-mask FLOPs) & % bf16 tensor peak; decode HBM GB/s",
+        def tf_frac(x):
+            return None if x is None else [r4(x["value"]), r4(x["roofline"]["frac"])]
+
+        summary = {"headline": tf_frac({"value": value, "roofline": roofline}) if value is not None else None,
+                   "headline_spread_pct": r4(repeats["spread_pct"]) if repeats else None,
+                   "cold_l2": tf_frac(cold), "e2e_tflops": r4(e2e["value"]) if e2e else None,
+                   "bwd": tf_frac(bwd), "fp8": tf_frac(fp8),
+                   "fp8_quantize_ms": r4(fp8["quantize_ms_per_step"]) if fp8 else None,
+                   "decode_gbs": tf_frac(decode), "decode_paged_gbs": tf_frac(decode_paged),
+                   "extra": {n: tf_frac(x) for n, x in extra.items()}}
+        if cpu:
+            summary["cpu"] = {"all_cores_tflops": r4(cpu["value"]), "one_core_tflops": r4(cpu["per_core"]["value"]),
+                              "cores": cpu["cores"]}
+            for n, x in cpu["configs"].items():
+                summary["cpu"][n] = ({"gbs": r4(x["gbs"]), "full_s_extrap": r4(x["extrapolated_full_run_s"])}
+                                     if "gbs" in x else
+                                     {"tflops": r4(x["tflops"]), "full_s_extrap": r4(x["extrapolated_full_run_s"])})
+        line = {"metric": METRIC,
                 "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
                 "config": {**w.describe(), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                           "l2": "inputs 201 MB (Q+K+V) > 126 MB L2, no flush",
+                           "l2": "inputs 201 MB (Q+K+V) > 126 MB L2, no flush (cold_l2: flushed)",
                            "kv_tiles_visited_per_head": counts["visited"],
                            "kv_tiles_total_per_head": counts["total"]},
-                "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
-                "clocks": clocks, "bwd": bwd, "fp8": fp8, "decode": decode, "decode_paged": decode_paged, "extra": extra,
-                "cpu_baseline": cpu}
+                "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps, "repeats": repeats,
+                "cold_l2": cold, "clocks": clocks, "decode": decode, "decode_paged": decode_paged,
+                "bwd": bwd, "fp8": fp8, "extra": extra, "cpu_baseline": cpu,
+                "summary": summary}
         print(json.dumps(line), flush=True)
 
 
@@ -537,6 +773,11 @@ def main():
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-full", action="store_true",
+                    help="CPU baseline on two full heads + 4096 rows of every other head, and every decode slice")
+    ap.add_argument("--sweep", action="store_true",
+                    help="sequence x window x batch matrix of the sliding-window page (one JSON line per point)")
+    ap.add_argument("--sweep-heads", type=int, default=32)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -33,7 +33,9 @@
  * is device memory owned by the caller, valid until the enqueued work is done.
  * Calls enqueue asynchronously on `stream` (a cudaStream_t, NULL = the legacy
  * default stream) and return once enqueued; the library allocates no device
- * memory.  Calls are thread-safe.  Library-owned state: a static decode
+ * memory.  Calls are thread-safe, with one exception: attn_decode_splitkv_noalloc
+ * calls that overlap on one device share its scratch and race (see there).
+ * Library-owned state: a static decode
  * scratch (attn_decode_splitkv_noalloc), 64 static work counters of the packed
  * prefill (attn_fwd_varlen), and, from the first attn_fwd_host call on a
  * device, three streams and eight events of that device.
@@ -235,6 +237,9 @@ int attn_fp8_ld(int Lk);
  *              ld = attn_fp8_ld(L), columns >= L written as 0 (transpose = 1)
  *   descale    device, fp32 [B*H] (written)
  * B*H <= 65535.  Four kernels (and a memset of descale) are enqueued.
+ * x must be finite: a NaN or an infinity in a head leaves that head's codes
+ * and descale undefined (no status is recorded), and so the FP8 forward's
+ * output for that head.
  */
 int attn_quantize_fp8(const void* x, void* codes, float* descale, int B, int H, int L, int d,
                       int transpose, void* stream);
@@ -382,7 +387,9 @@ int fattn_device_status(void* stream);
 
 /*
  * fattn_debug_inject_stall -- test hook for the failure path.  With on != 0
- * the next attn_fwd / attn_fwd_counted launch (only that one) leaves the
+ * the next bf16 prefill kernel launch of any kind, from any thread (attn_fwd,
+ * attn_fwd_counted, attn_fwd_varlen*, or one chunk of attn_fwd_host; only that
+ * one launch; the flag is process-wide; the FP8 forward ignores it) leaves the
  * first K tile of CTA 0 undelivered: nothing is loaded and nothing faults,
  * the waits that depend on it run out their time limit (about 2 s), and the
  * kernel records FATTN_ERR_TIMEOUT in the device status word, drains its

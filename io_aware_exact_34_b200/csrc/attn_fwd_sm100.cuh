@@ -360,18 +360,8 @@ __device__ __forceinline__ RowPlan row_plan(const FwdParams& p, int item, int t,
 // Exponentials of one 128-score row: p_c = 2^(s_c * c_log2 - m_safe), packed
 // to bf16 pairs in pk (key 2i in the low half of pk[i / 32][i % 32]); returns
 // the fp32 row sum of the p_c.  Scores are scaled and shifted in packed f32x2
-// FMAs.  On tiles with no masked position (kUnmasked) one pair in every
-// kPolyExp2Every goes through exp2_poly_pair on the FMA pipe, the rest through
-// the MUFU ex2; masked tiles use ex2 only, so masked scores (-inf) give
-// exactly 0.  Measured on B200 at d = 128 the MUFU is not the limit (any
-// polynomial share was slower), so the default share is zero.
-#ifndef FATTN_POLY_EXP2_EVERY
-#define FATTN_POLY_EXP2_EVERY 0
-#endif
-constexpr int kPolyExp2Every = FATTN_POLY_EXP2_EVERY;
-constexpr int kPolyExp2Mod = kPolyExp2Every > 0 ? kPolyExp2Every : 1;
-
-template <bool kUnmasked>
+// FMAs, exponentials on the MUFU (ex2.approx); masked scores (-inf) give
+// exactly 0.
 __device__ __forceinline__ float softmax_tile_probs(const uint32_t (&sr)[4][32], uint32_t (&pk)[2][32], float c_log2,
                                                     float m_safe) {
     const uint64_t scale2 = f2_pack(c_log2, c_log2);
@@ -382,14 +372,9 @@ __device__ __forceinline__ float softmax_tile_probs(const uint32_t (&sr)[4][32],
         const int c = 2 * i;
         const uint64_t s2 = f2_pack(__uint_as_float(sr[c >> 5][c & 31]), __uint_as_float(sr[c >> 5][(c & 31) + 1]));
         const uint64_t x2 = f2_fma(s2, scale2, shift2);
-        uint64_t p2;
-        if (kUnmasked && kPolyExp2Every > 0 && (i % kPolyExp2Mod) == kPolyExp2Mod - 1) {
-            p2 = exp2_poly_pair(x2);
-        } else {
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            p2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
-        }
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        const uint64_t p2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
         sum2[i & 3] = f2_add(sum2[i & 3], p2);
         float p0, p1;
         f2_unpack(p2, p0, p1);
@@ -760,12 +745,7 @@ __global__ void __launch_bounds__(384, 1)
                     tmem_st32(taddr_s, pk8);
                 } else {
                     uint32_t pk[2][32];
-                    float rowsum;
-                    if (full_tile)
-                        rowsum = softmax_tile_probs<true>(sr, pk, c_log2, m_safe);
-                    else
-                        rowsum = softmax_tile_probs<false>(sr, pk, c_log2, m_safe);
-                    l += rowsum;
+                    l += softmax_tile_probs(sr, pk, c_log2, m_safe);
                     tmem_st32(taddr_s, pk[0]);
                     tmem_st32(taddr_s + 32, pk[1]);
                 }

@@ -317,44 +317,10 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     return d;
 }
 
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
-}
-
-// 2^x for a pair of finite x <= 126 on the FMA pipe instead of the MUFU:
-// x = j + f with j = round(x) (by adding 1.5 * 2^23, whose low mantissa bits
-// then hold j) and f in [-0.5, 0.5]; 2^f by a cubic fitted here to minimise
-// the relative error on that interval (Lawson-weighted least squares: max
-// relative error 7.5e-5 in fp32, far below the 2^-9 rounding of bf16 P);
-// 2^j by adding j to the exponent field.  Inputs below -125 are clamped to
-// -125 (result 2^-125 instead of a smaller number), so callers only use it
-// where every input is an allowed score and the row sum is at least 1.
-__device__ __forceinline__ uint64_t exp2_poly_pair(uint64_t x) {
-    const uint64_t magic = 0x4B4000004B400000ull;  // 1.5 * 2^23, twice
-    const uint64_t c3 = 0x3D61FB813D61FB81ull;     // 0.05517149
-    const uint64_t c2 = 0x3E786F003E786F00ull;     // 0.24261093
-    const uint64_t c1 = 0x3F31798D3F31798Dull;     // 0.69326097
-    const uint64_t c0 = 0x3F7FFB493F7FFB49ull;     // 0.99992806
-    float x0, x1;
-    f2_unpack(x, x0, x1);
-    x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-    const uint64_t t = f2_add(x, magic);
-    const uint64_t f = f2_sub(x, f2_sub(t, magic));
-    uint64_t p = f2_fma(c3, f, c2);
-    p = f2_fma(p, f, c1);
-    p = f2_fma(p, f, c0);
-    const uint32_t t0 = static_cast<uint32_t>(t), t1 = static_cast<uint32_t>(t >> 32);
-    const uint32_t p0 = static_cast<uint32_t>(p), p1 = static_cast<uint32_t>(p >> 32);
-    const uint32_t r0 = p0 + (t0 << 23), r1 = p1 + (t1 << 23);
-    return (static_cast<uint64_t>(r1) << 32) | r0;
 }
 
 // Four floats rounded to e4m3 (nearest, ties to even, saturating at 448) in

@@ -60,6 +60,9 @@ WORKLOADS = {
     # causal prefill 4 x 16 x 4096, d = 128
     "causal_4k": Workload("causal_4k", "prefill", 4, 16, 4096, 4096, 128, "bf16",
                           causal=True, seed=2),
+    # the same causal prefill at head dim 64
+    "causal_4k_d64": Workload("causal_4k_d64", "prefill", 4, 16, 4096, 4096, 64, "bf16",
+                              causal=True, seed=8),
     # sliding window n = 32768, bidirectional |i - j| <= 2048
     "window_bidir_32k": Workload("window_bidir_32k", "prefill", 1, 32, 32768, 32768, 128,
                                  "bf16", window_left=2048, window_right=2048, seed=3),

@@ -167,24 +167,32 @@ def test_no_device_status_error(fl):
 
 # ------------------------------------------------------------------ full-size workloads
 
-def test_causal_4k_full(fl, oracle):
-    """Causal prefill 4 x 16 x 4096, d = 128: every row against the oracle."""
-    w = synth.WORKLOADS["causal_4k"]
+@pytest.mark.parametrize("name", ["causal_4k", "causal_4k_d64"])
+def test_causal_4k_full(fl, oracle, name):
+    """Causal prefill 4 x 16 x 4096 at d = 128 and d = 64: every row against
+    the oracle."""
+    w = synth.WORKLOADS[name]
     q, k, v = synth.make_inputs(w)
     o, lse = _run_bf16(fl, q, k, v, w.scale, w.causal, w.window_left, w.window_right)
     o_ref, lse_ref = oracle.attn(q, k, v, w.scale, w.causal, w.window_left, w.window_right)
-    compare(o, lse, o_ref, lse_ref, BF16_O_MAXABS, BF16_O_RELL2, label="causal_4k")
+    compare(o, lse, o_ref, lse_ref, BF16_O_MAXABS, BF16_O_RELL2, label=name)
 
 
 @pytest.mark.parametrize("name", ["window_bidir_32k", "window_causal_32k", "causal_64k_qscale"])
 def test_long_workloads_sampled(fl, oracle, name):
     """Sliding-window and long causal workloads at full size: the GPU runs
     the whole problem; the oracle checks one full head plus stratified rows of
-    every other head (first / last rows, tile and window edges, random)."""
+    every other head (first / last rows, tile and window edges, random).  For
+    the long causal workload with per-head query factors the full head is the
+    one with the largest factor, whose scores spread widest (the factor is
+    read back as the RMS of the head's Q, 8.4M draws)."""
     w = synth.WORKLOADS[name]
     q, k, v = synth.make_inputs(w)
     o, lse = _run_bf16(fl, q, k, v, w.scale, w.causal, w.window_left, w.window_right)
-    rows = synth.sample_rows(w, n_random=24, seed=7, full_heads=[(0, w.H - 1)] if w.Lq <= 32768 else [])
+    head = w.H - 1
+    if w.q_head_scale is not None:
+        head = int(q.float().pow(2).mean(dim=(0, 2, 3)).argmax())
+    rows = synth.sample_rows(w, n_random=24, seed=7, full_heads=[(0, head)])
     ro, rl = oracle.attn_rows(q, k, v, rows, w.scale, w.causal, w.window_left, w.window_right)
     r = rows.numpy()
     compare(o[r[:, 0], r[:, 1], r[:, 2]], lse[r[:, 0], r[:, 1], r[:, 2]], ro, rl,

@@ -5,16 +5,16 @@ is part of the library, so a caller that only owns its inputs and outputs (a
 plugin handed buffers by its host application, a service under a fixed memory
 budget) can run split-KV decode without a workspace.  These checks call it
 through the C ABI and compare it with attn_decode_splitkv, which takes a
-caller workspace, on two calls in a row with different shapes (the second call
-must not depend on what the first left in the shared scratch).  The file sorts
-last so that a run stopping at the first failure has run every other test.
+caller workspace, bit for bit on calls in a row with different shapes (a call
+must not depend on what the one before left in the shared scratch), and with
+the fp64 oracle.  The file sorts last so that a run stopping at the first
+failure has run every other test.
 """
-import numpy as np
 import pytest
 import torch
 
 from io_aware_exact_34_b200 import synth
-from tests._compare import BF16_O_MAXABS, LSE_ABS
+from tests._compare import BF16_O_MAXABS, BF16_O_RELL2, compare
 
 pytestmark = pytest.mark.gpu
 
@@ -40,17 +40,29 @@ def _inputs(B, H, Lk, d, seed):
 
 
 def test_noalloc_decode_matches_workspace_decode(fl):
-    for B, H, Lk, d, S, seed in [(6, 8, 5000, 128, 16, 21), (3, 4, 700, 64, 5, 22)]:
+    # Both entry points run the same split and merge kernels with the same
+    # split count, so their outputs must be identical bit for bit; a partial
+    # left in the shared scratch by the previous call would show up here.
+    # num_splits = 0 lets both pick the split count themselves.
+    for B, H, Lk, d, S, seed in [(6, 8, 5000, 128, 16, 21), (3, 4, 700, 64, 5, 22), (4, 8, 3000, 128, 0, 23)]:
         q, k, v, seqlens = _inputs(B, H, Lk, d, seed)
         o_ref, lse_ref = fl.attn_decode_splitkv(q, k, v, seqlens_k=seqlens, num_splits=S)
         o, lse = fl.attn_decode_splitkv_noalloc(q, k, v, seqlens_k=seqlens, num_splits=S)
         torch.cuda.synchronize()
-        o_ref, o = o_ref.float().cpu().numpy(), o.float().cpu().numpy()
-        lse_ref, lse = lse_ref.cpu().numpy(), lse.cpu().numpy()
-        assert np.abs(o - o_ref).max() <= BF16_O_MAXABS
-        empty = np.isneginf(lse_ref)
-        assert np.array_equal(np.isneginf(lse), empty)
-        assert np.abs(lse[~empty] - lse_ref[~empty]).max() <= LSE_ABS
+        assert torch.equal(o, o_ref)
+        assert torch.equal(lse, lse_ref)
+
+
+def test_noalloc_decode_matches_oracle(fl, oracle):
+    # the same check against the fp64 oracle directly, at the bars of the
+    # other decode tests
+    B, H, Lk, d = 3, 4, 2500, 128
+    q, k, v, seqlens = _inputs(B, H, Lk, d, 31)
+    o, lse = fl.attn_decode_splitkv_noalloc(q, k, v, seqlens_k=seqlens, num_splits=0)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attn(q.cpu(), k.cpu(), v.cpu(), d ** -0.5, seqlens_k=seqlens.cpu().numpy())
+    compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref[..., 0], BF16_O_MAXABS, BF16_O_RELL2,
+            label="noalloc decode")
 
 
 def test_noalloc_rejects_more_than_its_scratch(fl):
