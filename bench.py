@@ -687,7 +687,7 @@ def run_ours(args, world, rank, local):
 
     # ---------------------------------------------------------------- other prefill workloads
     extra = {}
-    if not args.no_extra:
+    if not args.no_extra and not args.no_d64:
         extra[HEADLINE_D64] = prefill_line(world, rank, dev, fattn, peaks, peak_src, HEADLINE_D64,
                                            max(3, min(args.steps, 20)))
     if not args.no_extra and not args.no_windows:
@@ -769,6 +769,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-windows", action="store_true", help="skip the window and 64K lines (keeps varlen)")
     ap.add_argument("--no-varlen", action="store_true", help="skip the packed varlen line")
+    ap.add_argument("--no-d64", action="store_true", help="skip the d = 64 prefill line")
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

@@ -36,9 +36,12 @@
  * memory.  Calls are thread-safe, with one exception: attn_decode_splitkv_noalloc
  * calls that overlap on one device share its scratch and race (see there).
  * Library-owned state: a static decode
- * scratch (attn_decode_splitkv_noalloc), 64 static work counters of the packed
- * prefill (attn_fwd_varlen), and, from the first attn_fwd_host call on a
- * device, three streams and eight events of that device.
+ * scratch (attn_decode_splitkv_noalloc), 64 static work counters from which
+ * the prefill kernels (attn_fwd*, attn_fwd_varlen*, attn_fwd_fp8*) deal their
+ * work items (each launch zeroes one with a 4-byte cudaMemsetAsync on its
+ * stream; more than 64 prefill launches in flight at once on one device
+ * would share counters), and, from the first attn_fwd_host call on a device,
+ * three streams and eight events of that device.
  *
  * Errors.  Every entry point returns a fattn_status; nothing aborts or throws.
  * Argument checks run before any CUDA call, so a rejected call enqueues

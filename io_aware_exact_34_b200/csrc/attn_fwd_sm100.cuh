@@ -132,6 +132,8 @@ struct FwdParams {
     int causal, window_left, window_right;
     int n_pairs, n_items;
     int vl_order;  // packed batches: 1 = work items in the compacted VarlenOrder, dealt by sched_ctr
+    int dyn_deal;  // dense batches: 1 = work items in head groups, dealt by sched_ctr
+    int group_heads;  // dense batches: heads per group of the dealt order (their K and V fit L2)
     unsigned int* sched_ctr;  // zeroed before the launch; the next slot to deal
     int o_vec32;   // O's base is 32-byte aligned: the epilogue writes 32-byte pieces of each row
     int inject_stall;  // test hook: CTA 0 never delivers its first K tile
@@ -184,6 +186,25 @@ struct PairTiles {
     int lo_t[2], hi_t[2];
     int lo, hi;  // union range
 };
+
+// Slot of the dealt dense order -> item index (pair-major: item =
+// (n_pairs - 1 - pair) * B*H + bh), or -1 past the last slot.  The dealt
+// order takes the heads in groups of group_heads (the last group may be
+// smaller) and, inside a group, pair indices descending, then heads: the
+// items in flight at any time read the K and V of few heads, which stay in
+// L2, and a CTA that drew short items takes more of them.
+__device__ __forceinline__ int dense_slot_item(const FwdParams& p, int slot) {
+    if (slot < 0 || slot >= p.n_items) return -1;
+    const int BH = p.B * p.H;
+    const int G = p.group_heads;
+    const int per_group = p.n_pairs * G;
+    const int g = slot / per_group;
+    const int r = slot - g * per_group;
+    const int gs = BH - g * G < G ? BH - g * G : G;
+    const int pair = p.n_pairs - 1 - r / gs;
+    const int bh = g * G + r % gs;
+    return (p.n_pairs - 1 - pair) * BH + bh;
+}
 
 __device__ __forceinline__ int snake_item(int round, int cta, int grid) {
     // Work items are ordered longest first; alternating the direction of
@@ -450,7 +471,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t p_ready0 = s_full0 + 16;
     const uint32_t o_full0 = p_ready0 + 16;
     const uint32_t drain_bar = o_full0 + 16;
-    const uint32_t item_full0 = drain_bar + 8;    // [2]: the producer dealt an item (packed batches)
+    const uint32_t item_full0 = drain_bar + 8;    // [2]: the producer dealt an item (dynamic deal)
     const uint32_t item_empty0 = item_full0 + 16;  // [2]: the MMA thread and the 8 softmax warps read it
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + T::SMEM_MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + T::SMEM_MISC_OFF + 4);
@@ -458,6 +479,11 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t vo_s = base + T::SMEM_VL_OFF;
     const bool vl = kVarlen && p.vl_order;
     if (vl) varlen_order_build(p, reinterpret_cast<VarlenOrder*>(gbase + T::SMEM_VL_OFF));
+    // dynamic deal: the producer takes slots from sched_ctr and hands the items
+    // to the MMA thread and the softmax warps through a two-entry ring here
+    const bool dyn = kVarlen ? vl : p.dyn_deal != 0;
+    const uint32_t item_ring_s =
+        kVarlen ? vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, item_slot)) : base + T::SMEM_MISC_OFF + 8;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -502,15 +528,16 @@ __global__ void __launch_bounds__(384, 1)
             bool ok = true;
             for (int round = 0; ok; ++round) {
                 int item;
-                if (vl) {
+                if (dyn) {
                     // deal: the next slot of the launch's counter, handed to the other roles
-                    item = varlen_slot_item(p, vo_s, static_cast<int>(atomicAdd(p.sched_ctr, 1u)));
+                    const int slot = static_cast<int>(atomicAdd(p.sched_ctr, 1u));
+                    item = kVarlen ? varlen_slot_item(p, vo_s, slot) : dense_slot_item(p, slot);
                     const int e = round & 1;
                     if (round >= 2) {
                         ok = mbar_wait(item_empty0 + 8 * e, ((round >> 1) - 1) & 1, abort_flag, status, -6);
                         if (!ok) break;
                     }
-                    sts_s32(vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, item_slot)) + 4u * e, item);
+                    sts_s32(item_ring_s + 4u * e, item);
                     mbar_arrive(item_full0 + 8 * e);
                 } else {
                     const int slot = snake_item(round, blockIdx.x, gridDim.x);
@@ -576,11 +603,11 @@ __global__ void __launch_bounds__(384, 1)
             bool ok = true;
             for (int round = 0; ok; ++round) {
                 int item;
-                if (vl) {
+                if (dyn) {
                     const int e = round & 1;
                     ok = mbar_wait(item_full0 + 8 * e, (round >> 1) & 1, abort_flag, status, -6);
                     if (!ok) break;
-                    item = lds_s32(vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, item_slot)) + 4u * e);
+                    item = lds_s32(item_ring_s + 4u * e);
                     mbar_arrive(item_empty0 + 8 * e);
                 } else {
                     const int slot = snake_item(round, blockIdx.x, gridDim.x);
@@ -676,12 +703,12 @@ __global__ void __launch_bounds__(384, 1)
         bool ok = true;
         for (int round = 0; ok; ++round) {
             int item;
-            if (vl) {
+            if (dyn) {
                 const int e = round & 1;
                 ok = mbar_wait(item_full0 + 8 * e, (round >> 1) & 1, abort_flag, status, -6);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
-                item = lds_s32(vo_s + static_cast<uint32_t>(offsetof(VarlenOrder, item_slot)) + 4u * e);
+                item = lds_s32(item_ring_s + 4u * e);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(item_empty0 + 8 * e);
             } else {

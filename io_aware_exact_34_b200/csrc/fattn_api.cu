@@ -63,7 +63,7 @@ std::atomic<int> g_inject_stall{0};
 __device__ __align__(256) float g_decode_noalloc_scratch[FATTN_DECODE_NOALLOC_SCRATCH_BYTES / sizeof(float)];
 void* g_noalloc_scratch_addr[kMaxDevices] = {};
 
-// Work counters of the packed prefill's dynamic deal: each launch takes the
+// Work counters of the prefill kernels' dynamic deal: each launch takes the
 // next of kSchedSlots counters (a host ticket) and zeroes it on its stream, so
 // launches in flight at the same time use different counters as long as
 // fewer than kSchedSlots of them overlap.
@@ -215,6 +215,29 @@ int encode_map_acc(CUtensorMap* map, float* base, int d, long long rows) {
     return r == CUDA_SUCCESS ? FATTN_OK : FATTN_ERR_CUDA;
 }
 
+// Dense prefill work order: heads in groups whose K and V together take at
+// most kL2GroupBytes (a part of the 126 MB L2, so the K/V tiles of the items in
+// flight are read from DRAM about once), dealt dynamically from a per-launch
+// counter zeroed on the stream.
+#ifndef FATTN_L2_GROUP_MB
+#define FATTN_L2_GROUP_MB 48
+#endif
+constexpr long long kL2GroupBytes = static_cast<long long>(FATTN_L2_GROUP_MB) << 20;
+
+int setup_dense_deal(FwdParams* p, long long BH, long long kv_bytes_per_head, void* stream) {
+    long long G = kv_bytes_per_head > 0 ? kL2GroupBytes / kv_bytes_per_head : BH;
+    G = G < 1 ? 1 : (G > BH ? BH : G);
+    p->dyn_deal = 1;
+    p->group_heads = static_cast<int>(G);
+    const int st = sched_counter(&p->sched_ctr);
+    if (st != FATTN_OK) return st;
+    if (cudaMemsetAsync(p->sched_ctr, 0, sizeof(unsigned int), static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return FATTN_ERR_CUDA;
+    }
+    return FATTN_OK;
+}
+
 template <int D, bool kVarlen>
 constexpr int fwd_smem_bytes() {
     return FwdTraits<D, false, kVarlen>::SMEM_BYTES;
@@ -262,9 +285,11 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.window_right = wr < 0 ? -1 : wr;
     p.n_pairs = static_cast<int>(n_pairs);
     p.n_items = static_cast<int>(n_items);
-    p.inject_stall = g_inject_stall.exchange(0);
     p.cu_q = p.cu_k = nullptr;
     p.total_q = p.total_k = 0;
+    st = setup_dense_deal(&p, BH, 2LL * Lk * d * 2, stream);
+    if (st != FATTN_OK) return st;
+    p.inject_stall = g_inject_stall.exchange(0);
     const int grid = static_cast<int>(n_items < di.num_sms ? n_items : di.num_sms);
     return launch_prefill_kernel<false>(mq, mk, mv, p, d, grid, static_cast<cudaStream_t>(stream));
 }
@@ -462,6 +487,8 @@ int launch_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float*
     p.q_descale = qd;
     p.k_descale = kd;
     p.v_descale = vd;
+    st = setup_dense_deal(&p, BH, 2LL * Lk * d, stream);
+    if (st != FATTN_OK) return st;
     const int grid = static_cast<int>(n_items < di.num_sms ? n_items : di.num_sms);
     attn_fwd_sm100_kernel<128, false, true><<<grid, FwdTraits<128, true>::THREADS, FwdTraits<128, true>::SMEM_BYTES,
                                                static_cast<cudaStream_t>(stream)>>>(mq, mk, mv, p);
