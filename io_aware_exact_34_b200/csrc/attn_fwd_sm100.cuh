@@ -33,10 +33,11 @@
 // FP8 instantiation (kFp8): Q, K are e4m3 [B,H,L,128] and V is e4m3 stored
 // transposed, [B,H,128,ldv], so both products read K-major operands; one fp32
 // descale per (b,h) for each of Q, K, V.  S = Q K^T and O += P V run as
-// kind::f8f6f4 MMAs (32 elements of K per instruction).  The running max is
-// exact (no slack) and p = 2^(x - m + 8) <= 2^8 is rounded to e4m3 before the
-// P V product, so typical probabilities sit in e4m3's normal range; l sums the
-// unrounded p; O = vd * acc / l and LSE = ln2 (m + log2 l - 8).  This is the
+// kind::f8f6f4 MMAs (32 elements of K per instruction).  The reference max
+// moves only when a tile's max passes it by more than kFp8Slack, and
+// p = 2^(x - m + 8 - kFp8Slack) <= 2^8 is rounded to e4m3 before the P V
+// product, so typical probabilities sit in e4m3's normal range; l sums the
+// unrounded p; O = vd * acc / l and LSE = ln2 (m + log2 l - 8 + kFp8Slack).  This is the
 // FP8 path FlashAttention-3 is named for in "FlashAttention 深度解析" §4,
 // taken on the tiled recurrence above.
 #pragma once
@@ -51,6 +52,10 @@
 namespace fattn {
 
 constexpr float kRescaleSlack = 8.0f;
+// FP8: the reference moves once a tile's max passes it by more than 4 (log2
+// units), and p = 2^(x - m + 8 - 4) <= 2^8 stays inside e4m3's range, with
+// typical probabilities in its normal range (reading R13).
+constexpr float kFp8Slack = 4.0f;
 
 // Work order of packed variable-length batches.  The dense item space (pair
 // index descending, then sequence, then head) holds an item for every pair
@@ -407,8 +412,8 @@ __device__ __forceinline__ float softmax_tile_probs(const uint32_t (&sr)[4][32],
     return lo + hi;
 }
 
-// FP8 variant: p_c = 2^(s_c * c_log2 - m_shift) (m_shift = m_safe - 8, so
-// p_c <= 2^8), rounded to e4m3 four to a word (key 4i in the low byte of
+// FP8 variant: p_c = 2^(s_c * c_log2 - m_shift) (m_shift = m_safe - 8 +
+// kFp8Slack, so p_c <= 2^8), rounded to e4m3 four to a word (key 4i in the low byte of
 // pk[i]); returns the fp32 sum of the unrounded p_c.  Masked scores (-inf)
 // give exactly 0.
 __device__ __forceinline__ float softmax_tile_probs_fp8(const uint32_t (&sr)[4][32], uint32_t (&pk)[32], float c_log2,
@@ -698,7 +703,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t taddr_s = tmem + lane_off + T::tm_s(t);
         const uint32_t taddr_o = tmem + lane_off + T::tm_o(t);
         const uint32_t s_full = s_full0 + 8 * t, p_ready = p_ready0 + 8 * t, o_full = o_full0 + 8 * t;
-        constexpr float slack = kFp8 ? 0.0f : kRescaleSlack;
+        constexpr float slack = kFp8 ? kFp8Slack : kRescaleSlack;
         uint32_t s_phase = 0, o_phase = 0;
         bool ok = true;
         for (int round = 0; ok; ++round) {
@@ -768,7 +773,7 @@ __global__ void __launch_bounds__(384, 1)
                 const float m_safe = (m_used == -CUDART_INF_F) ? 0.f : m_used;
                 if constexpr (kFp8) {
                     uint32_t pk8[32];
-                    l += softmax_tile_probs_fp8(sr, pk8, c_log2, m_safe - 8.f);
+                    l += softmax_tile_probs_fp8(sr, pk8, c_log2, m_safe - (8.f - kFp8Slack));
                     tmem_st32(taddr_s, pk8);
                 } else {
                     uint32_t pk[2][32];
@@ -826,7 +831,8 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             if (rp.valid && p.lse)
-                p.lse[rp.lse_off] = l > 0.f ? (m_used + __log2f(l) - (kFp8 ? 8.f : 0.f)) * 0.6931471805599453f : -CUDART_INF_F;
+                p.lse[rp.lse_off] =
+                    l > 0.f ? (m_used + __log2f(l) - (kFp8 ? 8.f - kFp8Slack : 0.f)) * 0.6931471805599453f : -CUDART_INF_F;
             if (p.visited && quarter == 0 && lane == 0)
                 atomicAdd(p.visited, static_cast<unsigned long long>(rp.hi - rp.lo));
         }

@@ -189,18 +189,22 @@ void oracle_quantize_fp8(const void* x, int dtype, long long groups, long long g
 
 /*
  * FP8 forward by the steps of reading R13 on the tiled online softmax of
- * [P2] §3.2, one query row at a time over key tiles of block_k keys:
+ * [P2] §3.2, one query row at a time over key tiles of block_k keys, with a
+ * reference max m that moves only when a tile's max exceeds it by more than
+ * `slack` (log2 units; 0 = the exact running max):
  *   x_j   = scale * qd * kd * (q8_i . k8_j) * log2(e)      (allowed keys)
- *   m'    = max(m, max_j x_j);  alpha = 2^(m - m');  l, acc *= alpha
- *   p_j   = 2^(x_j - m' + 8);   l += p_j
+ *   if max_j x_j > m + slack:  m' = max_j x_j;  alpha = 2^(m - m');  l, acc *= alpha
+ *   p_j   = 2^(x_j - m' + 8 - slack) <= 2^8;   l += p_j
  *   acc  += e4m3(p_j) * v8_j    (p_j itself when quantize_p == 0)
- * and at the end O = vd * acc / l, LSE = ln2 * (m + log2 l - 8).  q8, k8, v8
- * are e4m3 codes [B,H,L,d]; qd, kd, vd the per-(b,h) descales.  A row with no
- * allowed key gets O = 0 and LSE = -inf.
+ * and at the end O = vd * acc / l, LSE = ln2 * (m + log2 l - 8 + slack).
+ * Numerator and denominator share the reference, so without the rounding of
+ * p the result is exact attention for any slack.  q8, k8, v8 are e4m3 codes
+ * [B,H,L,d]; qd, kd, vd the per-(b,h) descales.  A row with no allowed key
+ * gets O = 0 and LSE = -inf.
  */
 void oracle_attn_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* qd, const float* kd,
                      const float* vd, double* o, double* lse, int B, int H, int Lq, int Lk, int d, double scale,
-                     int causal, int wl, int wr, int block_k, int quantize_p) {
+                     int causal, int wl, int wr, int block_k, int quantize_p, double slack) {
     const double LOG2E = 1.4426950408889634074;
     for (long long bh = 0; bh < static_cast<long long>(B) * H; ++bh) {
         std::vector<double> Kd(static_cast<size_t>(Lk) * d), Vd(static_cast<size_t>(Lk) * d);
@@ -227,7 +231,7 @@ void oracle_attn_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, co
                     mx = std::max(mx, x[t]);
                 }
                 if (mx == NEG_INF) continue;  /* no allowed key of this row in the tile */
-                if (mx > m) {
+                if (m == NEG_INF || mx > m + slack) {
                     const double alpha = m == NEG_INF ? 0.0 : std::exp2(m - mx);
                     l *= alpha;
                     for (int e = 0; e < d; ++e) acc[e] *= alpha;
@@ -235,7 +239,7 @@ void oracle_attn_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, co
                 }
                 for (int t = 0; t < n; ++t) {
                     if (!ok[t]) continue;
-                    const double p = std::exp2(x[t] - m + 8.0);
+                    const double p = std::exp2(x[t] - m + 8.0 - slack);
                     l += p;
                     const double pq = quantize_p ? e4m3_value(e4m3_round(p)) : p;
                     for (int e = 0; e < d; ++e) acc[e] += pq * Vd[(k0 + t) * d + e];
@@ -248,7 +252,7 @@ void oracle_attn_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, co
                 continue;
             }
             for (int e = 0; e < d; ++e) o[row * d + e] = static_cast<double>(vd[bh]) * acc[e] / l;
-            lse[row] = std::log(2.0) * (m + std::log2(l) - 8.0);
+            lse[row] = std::log(2.0) * (m + std::log2(l) - 8.0 + slack);
         }
     }
 }

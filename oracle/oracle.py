@@ -58,7 +58,7 @@ def _load():
             lib.oracle_e4m3_decode.argtypes = [u8p, ll, dp]
             lib.oracle_e4m3_encode.argtypes = [dp, ll, u8p]
             lib.oracle_quantize_fp8.argtypes = [vp, i, ll, ll, u8p, fp]
-            lib.oracle_attn_fp8.argtypes = [u8p, u8p, u8p, fp, fp, fp, dp, dp, i, i, i, i, i, d, i, i, i, i, i]
+            lib.oracle_attn_fp8.argtypes = [u8p, u8p, u8p, fp, fp, fp, dp, dp, i, i, i, i, i, d, i, i, i, i, i, d]
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_set_num_threads.argtypes = [i]
             _lib = lib
@@ -257,10 +257,17 @@ def quantize_fp8(x):
     return codes, desc
 
 
+# Reading R13: the FP8 recurrence keeps a reference max that moves only when a
+# tile's max passes it by more than FP8_SLACK (log2 units), and rounds
+# p = 2^(x - m + 8 - FP8_SLACK) <= 2^8 to e4m3.
+FP8_SLACK = 4.0
+
+
 def attn_fp8(q8, k8, v8, qd, kd, vd, scale, causal=False, window_left=-1, window_right=-1, block_k=128,
-             quantize_p=True):
+             quantize_p=True, slack=FP8_SLACK):
     """FP8 forward by its steps (e4m3 codes [B,H,L,d], per-(b,h) descales) ->
-    (O [B,H,Lq,d] float64, LSE [B,H,Lq] float64)."""
+    (O [B,H,Lq,d] float64, LSE [B,H,Lq] float64).  ``slack`` = 0 takes the exact
+    running max."""
     (q8, qp), (k8, kp), (v8, vp) = _u8(q8), _u8(k8), _u8(v8)
     (qd, qdp), (kd, kdp), (vd, vdp) = _f32(qd), _f32(kd), _f32(vd)
     B, H, Lq, d = q8.shape
@@ -269,7 +276,7 @@ def attn_fp8(q8, k8, v8, qd, kd, vd, scale, causal=False, window_left=-1, window
     lse = np.empty((B, H, Lq), np.float64)
     _load().oracle_attn_fp8(qp, kp, vp, qdp, kdp, vdp, _dptr(o), _dptr(lse), B, H, Lq, Lk, d, float(scale),
                             int(bool(causal)), int(window_left), int(window_right), int(block_k),
-                            int(bool(quantize_p)))
+                            int(bool(quantize_p)), float(slack))
     return o, lse
 
 

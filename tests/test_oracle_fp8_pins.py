@@ -3,7 +3,8 @@
 torch's float8_e4m3fn conversion and the format's closed forms, the
 per-head quantizer against the same conversion, the FP8 attention recurrence
 against the exact definition when P is not rounded, closed forms when every
-score is equal, and the rounding-error bound when it is."""
+score is equal, and the rounding-error bound when it is; for the exact
+running max (slack 0) and for reading R13's reference slack of 4."""
 import math
 
 import numpy as np
@@ -78,13 +79,18 @@ def _fp8_inputs(B, H, Lq, Lk, d, seed):
     return q8, k8, v8, qd, kd, vd
 
 
+@pytest.mark.parametrize("slack", [0.0, 4.0, 8.0])
 @pytest.mark.parametrize("Lq,Lk,causal,wl,wr,bk", [(40, 40, False, -1, -1, 16), (37, 53, True, -1, -1, 8),
                                                    (64, 64, False, 9, 4, 128), (50, 30, True, 5, 0, 7)])
-def test_fp8_recurrence_without_rounding_is_exact_attention(oracle, Lq, Lk, causal, wl, wr, bk):
-    """With P unrounded, the tiled FP8 recurrence (running max, rescale, the
-    2^8 factor, descales) is exact attention on the dequantized inputs."""
+def test_fp8_recurrence_without_rounding_is_exact_attention(oracle, Lq, Lk, causal, wl, wr, bk, slack):
+    """With P unrounded, the tiled FP8 recurrence (reference max with any
+    slack, rescale, the 2^(8 - slack) factor, descales) is exact attention on
+    the dequantized inputs: numerator and denominator share the reference."""
     q8, k8, v8, qd, kd, vd = _fp8_inputs(2, 2, Lq, Lk, 16, 3)
-    o, lse = oracle.attn_fp8(q8, k8, v8, qd, kd, vd, 0.25, causal, wl, wr, block_k=bk, quantize_p=False)
+    # scores spread widely enough that the reference moves at several tiles
+    q8 = oracle.e4m3_encode(oracle.e4m3_decode(q8) * 4.0)
+    o, lse = oracle.attn_fp8(q8, k8, v8, qd, kd, vd, 0.25, causal, wl, wr, block_k=bk, quantize_p=False,
+                             slack=slack)
     deq = lambda c, s: oracle.e4m3_decode(c) * s.astype(np.float64)[:, :, None, None]
     o_ref, lse_ref = oracle.attn(deq(q8, qd), deq(k8, kd), deq(v8, vd), 0.25, causal, wl, wr)
     fin = np.isfinite(lse_ref)
@@ -93,27 +99,30 @@ def test_fp8_recurrence_without_rounding_is_exact_attention(oracle, Lq, Lk, caus
     assert np.abs(lse[fin] - lse_ref[fin]).max() < 1e-10
 
 
-def test_fp8_equal_scores_give_exact_mean(oracle):
-    """All keys equal: every allowed p is exactly 2^8 (an e4m3 value), so even
-    with rounding O is the plain mean of the allowed dequantized V rows."""
+@pytest.mark.parametrize("slack", [0.0, 4.0])
+def test_fp8_equal_scores_give_exact_mean(oracle, slack):
+    """All keys equal: every allowed p is exactly 2^(8 - slack) (an e4m3
+    value), so even with rounding O is the plain mean of the allowed
+    dequantized V rows."""
     q8, _, v8, qd, kd, vd = _fp8_inputs(1, 2, 20, 20, 16, 4)
     k8 = np.broadcast_to(q8[:, :, :1], (1, 2, 20, 16)).copy()
-    o, lse = oracle.attn_fp8(q8, k8, v8, qd, kd, vd, 0.3, True, block_k=8, quantize_p=True)
+    o, lse = oracle.attn_fp8(q8, k8, v8, qd, kd, vd, 0.3, True, block_k=8, quantize_p=True, slack=slack)
     vdq = oracle.e4m3_decode(v8) * vd.astype(np.float64)[:, :, None, None]
     for i in range(20):
         assert np.abs(o[:, :, i] - vdq[:, :, : i + 1].mean(axis=2)).max() < 1e-13
 
 
-def test_fp8_rounding_error_within_bound(oracle):
+@pytest.mark.parametrize("slack", [0.0, 4.0])
+def test_fp8_rounding_error_within_bound(oracle, slack):
     """Rounding p (<= 2^8) to e4m3 changes each weight by at most 2^-4 of itself
     (3 mantissa bits, normal range) or 2^-10 absolute (subnormal range), so
     |O - O_unrounded| <= vd * max|v8| * (2^-4 + n * 2^-10 / l) per row."""
     q8, k8, v8, qd, kd, vd = _fp8_inputs(1, 2, 64, 64, 32, 5)
-    o_q, lse = oracle.attn_fp8(q8, k8, v8, qd, kd, vd, 0.5, False, quantize_p=True)
-    o_u, _ = oracle.attn_fp8(q8, k8, v8, qd, kd, vd, 0.5, False, quantize_p=False)
+    o_q, lse = oracle.attn_fp8(q8, k8, v8, qd, kd, vd, 0.5, False, quantize_p=True, slack=slack)
+    o_u, _ = oracle.attn_fp8(q8, k8, v8, qd, kd, vd, 0.5, False, quantize_p=False, slack=slack)
     vmax = np.abs(oracle.e4m3_decode(v8)).max(axis=(2, 3)) * vd
-    # l >= 2^8 (the row max contributes 2^8 exactly); n = 64 keys
-    bound = vmax[:, :, None] * (2.0 ** -4 + 64 * 2.0 ** -10 / 2.0 ** 8)
+    # l >= 2^(8 - slack) (the element that set the reference contributes at least that); n = 64 keys
+    bound = vmax[:, :, None] * (2.0 ** -4 + 64 * 2.0 ** -10 / 2.0 ** (8 - slack))
     err = np.abs(o_q - o_u).max(axis=3)
     assert np.all(err <= bound)
     assert err.max() > 0.0    # the rounding is really applied
