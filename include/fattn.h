@@ -191,10 +191,12 @@ int attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float
  * tensor cores' kind::f8f6f4 path ("FlashAttention 深度解析" §4 names
  * FlashAttention-3's FP8 path; this is the plain reading of it on the tiled
  * online softmax): S = Q K^T from the e4m3 codes with fp32 accumulation,
- * x = S * scale * q_descale * k_descale; against the exact running row max m,
- * p = 2^(x*log2e - m + 8) is rounded to e4m3 (nearest, ties to even) before
- * the P V product; l sums the unrounded p; O = v_descale * acc / l (bf16) and
- * LSE = ln2 (m + log2 l - 8) (fp32, natural log).  Mask as attn_fwd.
+ * x = S * scale * q_descale * k_descale; against a reference row max m that
+ * moves only when a tile's max passes it by more than 4 (log2 units; O and l
+ * are rescaled when it moves), p = 2^(x*log2e - m + 4) <= 2^8 is rounded to
+ * e4m3 (nearest, ties to even) before the P V product; l sums the unrounded
+ * p; O = v_descale * acc / l (bf16) and LSE = ln2 (m + log2 l - 4) (fp32,
+ * natural log).  Mask as attn_fwd.
  *
  *   q8         device, e4m3 codes [B,H,Lq,128]
  *   k8         device, e4m3 codes [B,H,Lk,128]
@@ -209,8 +211,9 @@ int attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float
  *
  * Accuracy against exact attention on the dequantized inputs: rounding p to
  * e4m3 changes each weight by at most 2^-4 of itself (2^-10 absolute below
- * e4m3's normal range), so a row's O moves by at most about
- * 2^-4 * max|v| and, for rows spread over many keys, far less.
+ * e4m3's normal range, against l >= 2^4), so a row's O moves by at most
+ * about 2^-4 * max|v| plus n * 2^-14 * max|v| for n keys, and, for rows
+ * spread over many keys, far less.
  */
 int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8,
                  const float* q_descale, const float* k_descale, const float* v_descale,
