@@ -17,7 +17,11 @@
 //   warps 4-7     softmax for Q tile 0 of the pair (one thread per row)
 //   warps 8-11    softmax for Q tile 1 of the pair
 // The two Q tiles share every K / V tile; while one softmax warpgroup turns
-// its S into P, the tensor core works on the other tile.
+// its S into P, the tensor core works on the other tile.  A work item is one
+// (batch, head, Q-tile pair); the producer deals items to the CTAs from a
+// per-launch counter, in head groups whose K and V fit a part of L2 (dense
+// batches) or in a compacted longest-first order (packed batches), and hands
+// each item to the MMA thread and the softmax warps through shared memory.
 //
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
 // P (bf16, two per 32-bit column) overwrites the first 64 columns of its S
