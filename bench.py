@@ -216,6 +216,50 @@ def timed(world, fn, steps, warmup):
     return max_over_ranks(world, start.elapsed_time(end) / steps)
 
 
+def timed_median(world, fn, steps, warmup, reps=3, gap_s=0.05, record=None):
+    """Median over `reps` timed regions of `steps` steps each.  Before each
+    region the device idles for `gap_s` of wall time and fn runs `warmup`
+    (then 3) untimed times.  Back-to-back regions of a long kernel drift down
+    to the power-capped clock within some tens of milliseconds; the idle gap
+    keeps every region a burst measurement, the regime of the measured burst
+    peak it is divided by, and the median keeps a region that caught a clock
+    transition out of the line.  `timed_sustained` gives the other regime."""
+    import torch
+    out = []
+    for r in range(reps):
+        torch.cuda.synchronize()
+        time.sleep(gap_s)
+        out.append(timed(world, fn, steps, warmup if r == 0 else 3))
+    if record is not None:
+        record.extend(out)
+    return statistics.median(out)
+
+
+SOAK_S = 0.5
+
+
+def timed_sustained(world, fn, steps, soak_s=SOAK_S):
+    """One region of `steps` steps timed right after fn has run back to back,
+    untimed, for `soak_s` of wall time: the clock the part settles at under its
+    power cap.  It is divided by the measured sustained peak."""
+    import torch
+    t_end = time.perf_counter() + soak_s
+    while time.perf_counter() < t_end:
+        for _ in range(10):
+            fn()
+        torch.cuda.synchronize()
+    return timed(world, fn, steps, 0)
+
+
+def sustained_entry(world, ms, flops, peaks, scale=1.0):
+    """The sustained figure of a TFLOP/s line against the measured sustained
+    bf16 peak (times `scale` for another dtype)."""
+    tf = flops / (ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"] * scale
+    return {"value": world * tf, "unit": "TFLOP/s", "ms_per_step": ms, "soak_s": SOAK_S,
+            "peak": peak, "frac": tf / peak, "peak_source": "bf16 dense, sustained" + (" x 2" if scale != 1.0 else "")}
+
+
 def timed_cold_l2(world, fn, steps, warmup, flush):
     """Average device ms per step of fn when every step starts with a cold L2:
     a write of `flush` (larger than L2) precedes each step outside the events
@@ -247,6 +291,20 @@ def tensor_roofline(achieved, peaks, peak_src, kernel, traffic, scale=1.0, scale
     src = f"{peak_src} bf16 dense (burst)" + scale_note
     return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": traffic, "peak_source": src, "kernel": kernel}
+
+
+def exp_roofline(achieved, peaks, peak_src, d):
+    """The exponential unit's ceiling on the same in-mask FLOPs: every allowed
+    pair needs one exp2, which runs on the special-function unit at 16 per
+    clock per SM, while the tensor core does 8192 dense bf16 FLOPs per clock
+    per SM.  At 4*d FLOPs per pair the exp rate caps the kernel at
+    16 * 4d / 8192 = d / 128 of the bf16 peak at the same clock, whatever the
+    MMA precision: half of it at d = 64, and the bf16 peak itself for the FP8
+    path at d = 128."""
+    peak = peaks["bf16_tflops"] * d / 128.0
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_source": f"{peak_src} bf16 dense (burst) x d/128 (16 exp2/clk/SM vs 8192 bf16 FLOP/clk/SM)",
+            "unit_bound": "MUFU ex2"}
 
 
 def r4(x):
@@ -435,12 +493,17 @@ def prefill_line(world, rank, dev, fl, peaks, peak_src, name, steps, warmup=3):
         fl.attn_fwd(eq, ek, ev, o=eo, lse=el, scale=we.scale, causal=we.causal,
                     window_left=we.window_left, window_right=we.window_right)
 
-    ems = timed(world, estep, steps, warmup)
+    regions = []
+    ems = timed_median(world, estep, steps, warmup, record=regions)
+    sms = timed_sustained(world, estep, steps)
     tf = f_e / (ems * 1e-3) / 1e12
     line = {"value": world * tf, "unit": "TFLOP/s", "ms_per_step": ems, "steps": steps,
             "roofline": tensor_roofline(tf, peaks, peak_src, PREFILL_KERNEL, recorded_traffic(PREFILL_KERNEL, name)),
             "kv_tiles_visited_per_head": c_e["visited"], "kv_tiles_total_per_head": c_e["total"],
-            "config": we.describe(), "gpu_launches": steps}
+            "config": we.describe(), "gpu_launches": steps, "regions_ms": regions,
+            "sustained": sustained_entry(world, sms, f_e, peaks)}
+    if we.d < 128:
+        line["exp_roofline"] = exp_roofline(tf, peaks, peak_src, we.d)
     del eq, ek, ev, eo, el
     torch.cuda.empty_cache()
     return line
@@ -513,7 +576,7 @@ def run_ours(args, world, rank, local):
         fattn.attn_fwd(q, k, v, o=o, lse=lse, scale=w.scale, causal=w.causal,
                        window_left=w.window_left, window_right=w.window_right)
 
-    ms, clocks, value, roofline, repeats, cold = float("nan"), None, None, None, None, None
+    ms, clocks, value, roofline, repeats, cold, sustained = float("nan"), None, None, None, None, None, None
     if not args.no_headline:
         def headline_regions():
             # the K-step region timed HEADLINE_REPEATS times; the median is the line's time
@@ -524,6 +587,7 @@ def run_ours(args, world, rank, local):
 
         if args.no_clocks:
             reps = headline_regions()
+            hs_ms = timed_sustained(world, step, args.steps, 1.0)
         else:
             with ClockSampler(local) as clk:
                 reps = headline_regions()
@@ -533,6 +597,8 @@ def run_ours(args, world, rank, local):
                     for _ in range(20):
                         step()
                     torch.cuda.synchronize()
+                # after a second of back-to-back work: the power-capped (sustained) regime
+                hs_ms = timed(world, step, args.steps, 0)
             clocks = clk.summary()
         ms = statistics.median(reps)
         value = world * flops / (ms * 1e-3) / 1e12
@@ -540,6 +606,8 @@ def run_ours(args, world, rank, local):
         roofline = tensor_roofline(achieved, peaks, peak_src, PREFILL_KERNEL, recorded_traffic(PREFILL_KERNEL, w.name))
         repeats = {"n": len(reps), "steps_each": args.steps, "ms_per_step": reps, "median": ms,
                    "min": min(reps), "max": max(reps), "spread_pct": 100.0 * (max(reps) - min(reps)) / ms}
+        sustained = sustained_entry(world, hs_ms, flops, peaks)
+        sustained["soak_s"] = 1.0
         # the same step with L2 flushed (a 256 MB write) before each launch
         flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
         cms = timed_cold_l2(world, step, args.steps, 3, flush)
@@ -583,7 +651,9 @@ def run_ours(args, world, rank, local):
                            window_right=w.window_right, dq=gq, dk=gk, dv=gv, workspace=gws)
 
         bsteps = max(3, min(args.steps, 20))
-        bms = timed(world, bstep, bsteps, 3)
+        bregions = []
+        bms = timed_median(world, bstep, bsteps, 3, record=bregions)
+        bsms = timed_sustained(world, bstep, bsteps)
         bflops = 2.5 * flops  # five products per allowed pair instead of two
         tf = bflops / (bms * 1e-3) / 1e12
         rl = tensor_roofline(tf, peaks, peak_src, "attn_bwd_sm100_kernel",
@@ -592,7 +662,8 @@ def run_ours(args, world, rank, local):
         bwd = {"metric": "attention bwd TFLOP/s (in-mask FLOPs: 10 d per allowed pair)", "value": world * tf,
                "unit": "TFLOP/s", "ms_per_step": bms, "steps": bsteps, "roofline": rl,
                "config": {**w.describe(), "pass": "backward with recomputation from LSE"},
-               "gpu_launches": 3 * bsteps}
+               "gpu_launches": 3 * bsteps, "regions_ms": bregions,
+               "sustained": sustained_entry(world, bsms, bflops, peaks)}
         del dout, gq, gk, gv, gws
         torch.cuda.empty_cache()
 
@@ -614,7 +685,9 @@ def run_ours(args, world, rank, local):
             fattn.attn_quantize_fp8(v, transpose=True, codes=vt8, descale=vs)
 
         fsteps = max(3, min(args.steps, 20))
-        fms = timed(world, fstep, fsteps, 3)
+        fregions = []
+        fms = timed_median(world, fstep, fsteps, 3, record=fregions)
+        fsms = timed_sustained(world, fstep, fsteps)
         qms = timed(world, qstep, 5, 3)
         tf = flops / (fms * 1e-3) / 1e12
         # nominal dense fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s) times the measured bf16 peak
@@ -622,6 +695,8 @@ def run_ours(args, world, rank, local):
                              recorded_traffic("attn_fwd_fp8", w.name), 2.0, " x 2 (nominal fp8/bf16 ratio)")
         fp8 = {"metric": "attention fwd TFLOP/s (in-mask FLOPs), e4m3 Q/K/V/P", "value": world * tf,
                "unit": "TFLOP/s", "ms_per_step": fms, "steps": fsteps, "roofline": rl,
+               "exp_roofline": exp_roofline(tf, peaks, peak_src, w.d),
+               "regions_ms": fregions, "sustained": sustained_entry(world, fsms, flops, peaks, 2.0),
                "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
                "quantize_ms_per_step": qms,
                "quantize_then_attend_tflops": world * flops / ((fms + qms) * 1e-3) / 1e12,
@@ -716,10 +791,13 @@ def run_ours(args, world, rank, local):
             fattn.attn_fwd_varlen(vq, vk, vv, cuq, cuk, max(lens), o=vo, lse=vl, causal=True)
 
         vsteps = max(3, min(args.steps, 10))
-        vms = timed(world, vstep, vsteps, 3)
+        vregions = []
+        vms = timed_median(world, vstep, vsteps, 3, record=vregions)
+        vsms = timed_sustained(world, vstep, vsteps)
         tf = f_v / (vms * 1e-3) / 1e12
         extra["varlen_causal_32seq"] = {
             "value": world * tf, "unit": "TFLOP/s", "ms_per_step": vms, "steps": vsteps,
+            "regions_ms": vregions, "sustained": sustained_entry(world, vsms, f_v, peaks),
             "roofline": tensor_roofline(tf, peaks, peak_src, PREFILL_KERNEL + "<128, true, false>",
                                         recorded_traffic(PREFILL_KERNEL, "varlen_causal_32seq")),
             "config": {"workload": "varlen_causal_32seq", "num_seqs": VARLEN_SEQS,
@@ -743,7 +821,12 @@ def run_ours(args, world, rank, local):
                    "bwd": tf_frac(bwd), "fp8": tf_frac(fp8),
                    "fp8_quantize_ms": r4(fp8["quantize_ms_per_step"]) if fp8 else None,
                    "decode_gbs": tf_frac(decode), "decode_paged_gbs": tf_frac(decode_paged),
-                   "extra": {n: tf_frac(x) for n, x in extra.items()}}
+                   "extra": {n: tf_frac(x) for n, x in extra.items()},
+                   "exp_frac": {n: r4(x["exp_roofline"]["frac"])
+                                for n, x in [("fp8", fp8), *extra.items()] if x and "exp_roofline" in x},
+                   "sustained": {n: [r4(x["sustained"]["value"]), r4(x["sustained"]["frac"])]
+                                 for n, x in [("headline", {"sustained": sustained}), ("bwd", bwd), ("fp8", fp8),
+                                              *extra.items()] if x and x.get("sustained")}}
         if cpu:
             summary["cpu"] = {"all_cores_tflops": r4(cpu["value"]), "one_core_tflops": r4(cpu["per_core"]["value"]),
                               "cores": cpu["cores"]}
@@ -760,6 +843,7 @@ def run_ours(args, world, rank, local):
                            "kv_tiles_visited_per_head": counts["visited"],
                            "kv_tiles_total_per_head": counts["total"]},
                 "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps, "repeats": repeats,
+                "sustained": sustained,
                 "cold_l2": cold, "clocks": clocks, "decode": decode, "decode_paged": decode_paged,
                 "bwd": bwd, "fp8": fp8, "extra": extra, "cpu_baseline": cpu,
                 "summary": summary}
