@@ -25,7 +25,13 @@
 //
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
 // P (bf16, two per 32-bit column) overwrites the first 64 columns of its S
-// tile and feeds the P.V MMA straight from TMEM.
+// tile and feeds the P.V MMA straight from TMEM, so a tile's next S waits for
+// its P.V product.  At d = 64 in bf16 the O tiles leave 128 columns free: P0
+// and P1 take [256,384), O0 and O1 move to [384,512), and a tile's next S is
+// issued as soon as its softmax warps have read the current S (s_free), so
+// the exponentials of one KV tile overlap the S product of the next; the
+// softmax waits for the previous P.V product (p_free) before it writes P or
+// rescales O.
 //
 // Exact rescale skipping: the running max used for the exponentials is only
 // raised when a new row max exceeds it by more than kRescaleSlack (log2
@@ -107,7 +113,15 @@ struct FwdTraits {
     static constexpr int SMEM_Q_OFF = 0;
     static constexpr int SMEM_RING_OFF = 2 * TILE_BYTES;
     static constexpr int SMEM_BAR_OFF = SMEM_RING_OFF + NSTAGE * TILE_BYTES;
-    static constexpr int NBAR = 2 + 2 * NSTAGE + 6 + 1 + 4;
+    // Decoupled P (bf16, d = 64): the two O tiles take 128 TMEM columns, so P
+    // gets columns of its own and a tile's next S = Q K^T is issued as soon as
+    // its softmax warps have read the current S into registers, while the
+    // exponentials of that S run.  At d = 128 S0, S1, O0, O1 fill TMEM and P
+    // overwrites its S tile, so the next S waits for the P V product.
+    static constexpr bool DEC = (D == 64) && !kFp8;
+    // q_full/empty, kv_full/empty[NSTAGE], s_full/p_ready/o_full[2], drain,
+    // item_full/empty[2]; decoupled: s_free[2], p_free[2]
+    static constexpr int NBAR = 2 + 2 * NSTAGE + 6 + 1 + 4 + (DEC ? 4 : 0);
     static constexpr int SMEM_MISC_OFF = SMEM_BAR_OFF + NBAR * 8;
     // packed batches: the VarlenOrder table after the misc words
     static constexpr int SMEM_VL_OFF = SMEM_MISC_OFF + 16;
@@ -125,8 +139,16 @@ struct FwdTraits {
     static constexpr uint32_t REGS_HIGH = 208;
     static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= THREADS * REGS_LAUNCH, "register split");
     static constexpr uint32_t TMEM_COLS = 512;
+    // S0, S1 [0, 256); decoupled: P0, P1 [256, 384) (bf16, two per column),
+    // O0, O1 [384, 512); otherwise O0, O1 [256, 256 + 2D) and P in its S tile
     __host__ __device__ static constexpr uint32_t tm_s(int t) { return static_cast<uint32_t>(t) * 128u; }
-    __host__ __device__ static constexpr uint32_t tm_o(int t) { return 256u + static_cast<uint32_t>(t) * D; }
+    __host__ __device__ static constexpr uint32_t tm_p(int t) {
+        return DEC ? 256u + static_cast<uint32_t>(t) * 64u : tm_s(t);
+    }
+    __host__ __device__ static constexpr uint32_t tm_o(int t) {
+        return (DEC ? 384u : 256u) + static_cast<uint32_t>(t) * D;
+    }
+    static_assert(!DEC || 384 + 2 * D <= 512, "decoupled TMEM layout");
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(!kFp8 || D == 128, "the FP8 path is built for d = 128");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory");
@@ -482,6 +504,8 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t drain_bar = o_full0 + 16;
     const uint32_t item_full0 = drain_bar + 8;    // [2]: the producer dealt an item (dynamic deal)
     const uint32_t item_empty0 = item_full0 + 16;  // [2]: the MMA thread and the 8 softmax warps read it
+    const uint32_t s_free0 = item_empty0 + 16;     // [2] decoupled: the softmax warps have read S out of TMEM
+    const uint32_t p_free0 = s_free0 + 16;         // [2] decoupled: the P V product that read P is done
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + T::SMEM_MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + T::SMEM_MISC_OFF + 4);
     int* status = &g_fattn_status;
@@ -510,6 +534,12 @@ __global__ void __launch_bounds__(384, 1)
         for (int e = 0; e < 2; ++e) {
             mbar_init(item_full0 + 8 * e, 1);
             mbar_init(item_empty0 + 8 * e, 9);
+        }
+        if constexpr (T::DEC) {
+            for (int t = 0; t < 2; ++t) {
+                mbar_init(s_free0 + 8 * t, 4);  // lane 0 of each of the tile's four softmax warps
+                mbar_init(p_free0 + 8 * t, 1);
+            }
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -609,6 +639,7 @@ __global__ void __launch_bounds__(384, 1)
             // FP8: V^T is K-major; bf16: V is MN-major (d contiguous)
             constexpr uint32_t idesc_pv = kFp8 ? idesc_e4m3_f32(128, D, 0, 0) : idesc_bf16_f32(128, D, 0, 1);
             uint32_t ring = 0, q_round = 0, p_cnt[2] = {0u, 0u};
+            [[maybe_unused]] uint32_t s_cnt[2] = {0u, 0u};  // decoupled: S products issued per tile
             bool ok = true;
             for (int round = 0; ok; ++round) {
                 int item;
@@ -635,62 +666,102 @@ __global__ void __launch_bounds__(384, 1)
                     const bool haveV = j > ts.lo;
                     const uint32_t rK = ring0 + 2u * static_cast<uint32_t>(j - ts.lo);
                     const uint32_t rV = rK - 1u;  // V tile of KV tile j-1
-                    if (haveK) ok = mbar_wait(kv_full0 + 8 * (rK % T::NSTAGE), (rK / T::NSTAGE) & 1u, abort_flag, status, -6);
-                    if (ok && haveV) ok = mbar_wait(kv_full0 + 8 * (rV % T::NSTAGE), (rV / T::NSTAGE) & 1u, abort_flag, status, -6);
-                    if (!ok) break;
-                    tc_fence_after_sync();
-                    for (int t = 0; t < 2 && ok; ++t) {
-                        // O_t += P_t V_{j-1}
-                        if (haveV && j - 1 >= ts.lo_t[t] && j - 1 < ts.hi_t[t]) {
+                    bool doS[2], doPV[2];
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        doS[t] = haveK && j >= ts.lo_t[t] && j < ts.hi_t[t];
+                        doPV[t] = haveV && j - 1 >= ts.lo_t[t] && j - 1 < ts.hi_t[t];
+                    }
+                    // S_t = Q_t K_j^T
+                    auto issue_s = [&](int t) {
+                        const uint32_t k_lo = sdesc_lo(sRing + (rK % T::NSTAGE) * T::TILE_BYTES, 16);
+                        const uint32_t q_lo = sdesc_lo(sQ + t * T::TILE_BYTES, 16);
+#pragma unroll
+                        for (int ks = 0; ks < T::KSTEPS_S; ++ks) {
+                            // 32 B along the swizzled row per step; every 128 B the next 16 KB column
+                            const uint32_t off = ((ks / 4) * T::CHUNK_BYTES + (ks % 4) * 32) >> 4;
+                            if constexpr (kFp8)
+                                mma_fp8_ss(tmem + T::tm_s(t), sdesc_from_lo(q_lo + off), sdesc_from_lo(k_lo + off),
+                                           idesc_s, ks > 0 ? 1u : 0u);
+                            else
+                                mma_bf16_ss(tmem + T::tm_s(t), sdesc_from_lo(q_lo + off), sdesc_from_lo(k_lo + off),
+                                            idesc_s, ks > 0 ? 1u : 0u);
+                        }
+                        mma_commit(s_full0 + 8 * t);
+                    };
+                    // O_t += P_t V_{j-1}
+                    auto issue_pv = [&](int t) {
+                        const uint32_t first = (j - 1 == ts.lo_t[t]) ? 1u : 0u;
+                        if constexpr (kFp8) {
+                            const uint32_t v_lo = sdesc_lo(sRing + (rV % T::NSTAGE) * T::TILE_BYTES, 16);
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks) {
+                                // 32 keys = 8 TMEM columns of packed P, 32 B along the V^T rows
+                                mma_fp8_ts(tmem + T::tm_o(t), tmem + T::tm_p(t) + ks * 8,
+                                           sdesc_from_lo(v_lo + ks * (32 >> 4)), idesc_pv, (first && ks == 0) ? 0u : 1u);
+                            }
+                        } else {
+                            const uint32_t v_lo = sdesc_lo(sRing + (rV % T::NSTAGE) * T::TILE_BYTES, T::CHUNK_BYTES);
+#pragma unroll
+                            for (int ks = 0; ks < 8; ++ks) {
+                                // 16 keys = 8 TMEM columns of packed P, 16 rows of 128 B further into the V tile
+                                mma_bf16_ts(tmem + T::tm_o(t), tmem + T::tm_p(t) + ks * 8,
+                                            sdesc_from_lo(v_lo + ks * (2048 >> 4)), idesc_pv,
+                                            (first && ks == 0) ? 0u : 1u);
+                            }
+                        }
+                        if (j - 1 == ts.hi_t[t] - 1) mma_commit(o_full0 + 8 * t);
+                    };
+                    if constexpr (T::DEC) {
+                        // S of both tiles first, each as soon as its softmax warps have read
+                        // the previous S; then the P V products of the previous KV tile
+                        if (haveK) ok = mbar_wait(kv_full0 + 8 * (rK % T::NSTAGE), (rK / T::NSTAGE) & 1u, abort_flag, status, -6);
+                        for (int t = 0; t < 2 && ok; ++t) {
+                            if (!doS[t]) continue;
+                            if (s_cnt[t] > 0) ok = mbar_wait(s_free0 + 8 * t, (s_cnt[t] - 1u) & 1u, abort_flag, status, -6);
+                            if (!ok) break;
+                            ++s_cnt[t];
+                            tc_fence_after_sync();
+                            issue_s(t);
+                        }
+                        if (!ok) break;
+                        if (haveK) {
+                            mma_commit(kv_empty0 + 8 * (rK % T::NSTAGE));
+                            if (j == ts.hi - 1) mma_commit(q_empty);
+                        }
+                        if (haveV) ok = mbar_wait(kv_full0 + 8 * (rV % T::NSTAGE), (rV / T::NSTAGE) & 1u, abort_flag, status, -6);
+                        for (int t = 0; t < 2 && ok; ++t) {
+                            if (!doPV[t]) continue;
                             ok = mbar_wait(p_ready0 + 8 * t, p_cnt[t] & 1u, abort_flag, status, -6);
                             ++p_cnt[t];
                             if (!ok) break;
                             tc_fence_after_sync();
-                            const uint32_t first = (j - 1 == ts.lo_t[t]) ? 1u : 0u;
-                            if constexpr (kFp8) {
-                                const uint32_t v_lo = sdesc_lo(sRing + (rV % T::NSTAGE) * T::TILE_BYTES, 16);
-#pragma unroll
-                                for (int ks = 0; ks < 4; ++ks) {
-                                    // 32 keys = 8 TMEM columns of packed P, 32 B along the V^T rows
-                                    mma_fp8_ts(tmem + T::tm_o(t), tmem + T::tm_s(t) + ks * 8,
-                                               sdesc_from_lo(v_lo + ks * (32 >> 4)), idesc_pv,
-                                               (first && ks == 0) ? 0u : 1u);
-                                }
-                            } else {
-                                const uint32_t v_lo = sdesc_lo(sRing + (rV % T::NSTAGE) * T::TILE_BYTES, T::CHUNK_BYTES);
-#pragma unroll
-                                for (int ks = 0; ks < 8; ++ks) {
-                                    // 16 keys = 16 rows of 128 B further into the V tile
-                                    mma_bf16_ts(tmem + T::tm_o(t), tmem + T::tm_s(t) + ks * 8,
-                                                sdesc_from_lo(v_lo + ks * (2048 >> 4)), idesc_pv,
-                                                (first && ks == 0) ? 0u : 1u);
-                                }
-                            }
-                            if (j - 1 == ts.hi_t[t] - 1) mma_commit(o_full0 + 8 * t);
+                            issue_pv(t);
+                            mma_commit(p_free0 + 8 * t);
                         }
-                        // S_t = Q_t K_j^T
-                        if (haveK && j >= ts.lo_t[t] && j < ts.hi_t[t]) {
-                            const uint32_t k_lo = sdesc_lo(sRing + (rK % T::NSTAGE) * T::TILE_BYTES, 16);
-                            const uint32_t q_lo = sdesc_lo(sQ + t * T::TILE_BYTES, 16);
-#pragma unroll
-                            for (int ks = 0; ks < T::KSTEPS_S; ++ks) {
-                                // 32 B along the swizzled row per step; every 128 B the next 16 KB column
-                                const uint32_t off = ((ks / 4) * T::CHUNK_BYTES + (ks % 4) * 32) >> 4;
-                                if constexpr (kFp8)
-                                    mma_fp8_ss(tmem + T::tm_s(t), sdesc_from_lo(q_lo + off), sdesc_from_lo(k_lo + off),
-                                               idesc_s, ks > 0 ? 1u : 0u);
-                                else
-                                    mma_bf16_ss(tmem + T::tm_s(t), sdesc_from_lo(q_lo + off), sdesc_from_lo(k_lo + off),
-                                                idesc_s, ks > 0 ? 1u : 0u);
+                        if (!ok) break;
+                        if (haveV) mma_commit(kv_empty0 + 8 * (rV % T::NSTAGE));
+                    } else {
+                        if (haveK) ok = mbar_wait(kv_full0 + 8 * (rK % T::NSTAGE), (rK / T::NSTAGE) & 1u, abort_flag, status, -6);
+                        if (ok && haveV) ok = mbar_wait(kv_full0 + 8 * (rV % T::NSTAGE), (rV / T::NSTAGE) & 1u, abort_flag, status, -6);
+                        if (!ok) break;
+                        tc_fence_after_sync();
+                        for (int t = 0; t < 2 && ok; ++t) {
+                            if (doPV[t]) {
+                                ok = mbar_wait(p_ready0 + 8 * t, p_cnt[t] & 1u, abort_flag, status, -6);
+                                ++p_cnt[t];
+                                if (!ok) break;
+                                tc_fence_after_sync();
+                                issue_pv(t);
                             }
-                            mma_commit(s_full0 + 8 * t);
+                            if (doS[t]) issue_s(t);
                         }
-                    }
-                    if (!ok) break;
-                    if (haveV) mma_commit(kv_empty0 + 8 * (rV % T::NSTAGE));
-                    if (haveK) {
-                        mma_commit(kv_empty0 + 8 * (rK % T::NSTAGE));
-                        if (j == ts.hi - 1) mma_commit(q_empty);
+                        if (!ok) break;
+                        if (haveV) mma_commit(kv_empty0 + 8 * (rV % T::NSTAGE));
+                        if (haveK) {
+                            mma_commit(kv_empty0 + 8 * (rK % T::NSTAGE));
+                            if (j == ts.hi - 1) mma_commit(q_empty);
+                        }
                     }
                 }
                 ring = ring0 + 2u * static_cast<uint32_t>(ts.hi - ts.lo);
@@ -706,9 +777,11 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t taddr_s = tmem + lane_off + T::tm_s(t);
         const uint32_t taddr_o = tmem + lane_off + T::tm_o(t);
+        const uint32_t taddr_p = tmem + lane_off + T::tm_p(t);
         const uint32_t s_full = s_full0 + 8 * t, p_ready = p_ready0 + 8 * t, o_full = o_full0 + 8 * t;
         constexpr float slack = kFp8 ? kFp8Slack : kRescaleSlack;
         uint32_t s_phase = 0, o_phase = 0;
+        [[maybe_unused]] uint32_t p_cnt = 0;  // decoupled: P tiles this warpgroup has written
         bool ok = true;
         for (int round = 0; ok; ++round) {
             int item;
@@ -756,6 +829,12 @@ __global__ void __launch_bounds__(384, 1)
                 tmem_wait_ld();
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) reg_fence(sr[q4]);
+                if constexpr (T::DEC) {
+                    // S is in registers: the next S of this tile may overwrite its columns
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(s_free0 + 8 * t);
+                }
                 const int k0 = j * 128;
                 const bool full_tile = k0 >= rp.full_lo && k0 + 127 <= rp.full_hi;
                 if (!full_tile) {
@@ -782,8 +861,19 @@ __global__ void __launch_bounds__(384, 1)
                 } else {
                     uint32_t pk[2][32];
                     l += softmax_tile_probs(sr, pk, c_log2, m_safe);
-                    tmem_st32(taddr_s, pk[0]);
-                    tmem_st32(taddr_s + 32, pk[1]);
+                    if constexpr (T::DEC) {
+                        // the P V product that read the previous P of this tile, and
+                        // accumulated into O, is done: P and O may be written
+                        if (p_cnt > 0) {
+                            ok = mbar_wait(p_free0 + 8 * t, (p_cnt - 1u) & 1u, abort_flag, status, -6);
+                            ok = __all_sync(0xffffffffu, ok);
+                            if (!ok) break;
+                            tc_fence_after_sync();
+                        }
+                        ++p_cnt;
+                    }
+                    tmem_st32(taddr_p, pk[0]);
+                    tmem_st32(taddr_p + 32, pk[1]);
                 }
                 if (__any_sync(0xffffffffu, resc)) {
                     const float a = resc ? alpha : 1.f;
