@@ -216,7 +216,11 @@ def timed(world, fn, steps, warmup):
     return max_over_ranks(world, start.elapsed_time(end) / steps)
 
 
-def timed_median(world, fn, steps, warmup, reps=3, gap_s=0.05, record=None):
+REGIONS = 3          # burst regions per secondary line (--regions)
+SUSTAINED = True     # time the sustained regime too (--no-sustained turns it off)
+
+
+def timed_median(world, fn, steps, warmup, reps=None, gap_s=0.05, record=None):
     """Median over `reps` timed regions of `steps` steps each.  Before each
     region the device idles for `gap_s` of wall time and fn runs `warmup`
     (then 3) untimed times.  Back-to-back regions of a long kernel drift down
@@ -225,6 +229,7 @@ def timed_median(world, fn, steps, warmup, reps=3, gap_s=0.05, record=None):
     peak it is divided by, and the median keeps a region that caught a clock
     transition out of the line.  `timed_sustained` gives the other regime."""
     import torch
+    reps = REGIONS if reps is None else reps
     out = []
     for r in range(reps):
         torch.cuda.synchronize()
@@ -241,8 +246,11 @@ SOAK_S = 0.5
 def timed_sustained(world, fn, steps, soak_s=SOAK_S):
     """One region of `steps` steps timed right after fn has run back to back,
     untimed, for `soak_s` of wall time: the clock the part settles at under its
-    power cap.  It is divided by the measured sustained peak."""
+    power cap.  It is divided by the measured sustained peak.  None when the
+    sustained regime is switched off."""
     import torch
+    if not SUSTAINED:
+        return None
     t_end = time.perf_counter() + soak_s
     while time.perf_counter() < t_end:
         for _ in range(10):
@@ -254,6 +262,8 @@ def timed_sustained(world, fn, steps, soak_s=SOAK_S):
 def sustained_entry(world, ms, flops, peaks, scale=1.0):
     """The sustained figure of a TFLOP/s line against the measured sustained
     bf16 peak (times `scale` for another dtype)."""
+    if ms is None:
+        return None
     tf = flops / (ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"] * scale
     return {"value": world * tf, "unit": "TFLOP/s", "ms_per_step": ms, "soak_s": SOAK_S,
@@ -598,7 +608,7 @@ def run_ours(args, world, rank, local):
                         step()
                     torch.cuda.synchronize()
                 # after a second of back-to-back work: the power-capped (sustained) regime
-                hs_ms = timed(world, step, args.steps, 0)
+                hs_ms = timed(world, step, args.steps, 0) if SUSTAINED else None
             clocks = clk.summary()
         ms = statistics.median(reps)
         value = world * flops / (ms * 1e-3) / 1e12
@@ -607,7 +617,8 @@ def run_ours(args, world, rank, local):
         repeats = {"n": len(reps), "steps_each": args.steps, "ms_per_step": reps, "median": ms,
                    "min": min(reps), "max": max(reps), "spread_pct": 100.0 * (max(reps) - min(reps)) / ms}
         sustained = sustained_entry(world, hs_ms, flops, peaks)
-        sustained["soak_s"] = 1.0
+        if sustained:
+            sustained["soak_s"] = 1.0
         # the same step with L2 flushed (a 256 MB write) before each launch
         flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
         cms = timed_cold_l2(world, step, args.steps, 3, flush)
@@ -867,6 +878,8 @@ def main():
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sustained", action="store_true", help="skip the sustained regions (profiling runs)")
+    ap.add_argument("--regions", type=int, default=3, help="burst regions per secondary line (median taken)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-full", action="store_true",
                     help="CPU baseline on two full heads + 4096 rows of every other head, and every decode slice")
@@ -876,6 +889,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    global REGIONS, SUSTAINED
+    REGIONS = max(1, args.regions)
+    SUSTAINED = not args.no_sustained
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
