@@ -108,14 +108,28 @@ def test_bf16_grid(fl, oracle, B, H, Lq, Lk, d, causal, wl, wr):
     compare(o, lse, o_ref, lse_ref, BF16_O_MAXABS, BF16_O_RELL2, label=f"bf16 {B,H,Lq,Lk,d,causal,wl,wr}")
 
 
-def test_bf16_large_scores_stress_rescale(fl, oracle):
+@pytest.mark.parametrize("d,causal,wl,wr", [(128, True, -1, -1), (64, True, -1, -1), (64, False, 300, 300),
+                                             (64, True, 700, 0)])
+def test_bf16_large_scores_stress_rescale(fl, oracle, d, causal, wl, wr):
     """Scores spread over a wide range (Q scaled by 6): the running-max
-    reference moves many times and the accumulator rescale path runs."""
-    q, k, v = synth.random_qkv(1, 4, 1024, 1024, 128, "bf16", seed=99)
+    reference moves many times and the accumulator rescale path runs (at
+    d = 64 after the wait for the previous P.V product, P having columns of
+    its own)."""
+    q, k, v = synth.random_qkv(1, 4, 1024, 1024, d, "bf16", seed=99 + d + max(wl, 0))
     q = (q.float() * 6.0).to(torch.bfloat16)
-    o, lse = _run_bf16(fl, q, k, v, 128 ** -0.5, True, -1, -1)
-    o_ref, lse_ref = oracle.attn(q, k, v, 128 ** -0.5, True)
-    compare(o, lse, o_ref, lse_ref, BF16_O_MAXABS, BF16_O_RELL2, label="rescale stress")
+    o, lse = _run_bf16(fl, q, k, v, d ** -0.5, causal, wl, wr)
+    o_ref, lse_ref = oracle.attn(q, k, v, d ** -0.5, causal, wl, wr)
+    compare(o, lse, o_ref, lse_ref, BF16_O_MAXABS, BF16_O_RELL2, label=f"rescale stress d={d} {causal,wl,wr}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_many_short_items(fl, oracle, d):
+    """Many work items per CTA (8 x 16 heads of 600 tokens, causal): every
+    item boundary hands S, P and O of both tiles over to the next item."""
+    q, k, v = synth.random_qkv(8, 16, 600, 600, d, "bf16", seed=400 + d)
+    o, lse = _run_bf16(fl, q, k, v, d ** -0.5, True, -1, -1)
+    o_ref, lse_ref = oracle.attn(q, k, v, d ** -0.5, True)
+    compare(o, lse, o_ref, lse_ref, BF16_O_MAXABS, BF16_O_RELL2, label=f"short items d={d}")
 
 
 def test_constant_v_rows(fl):
