@@ -131,12 +131,13 @@ struct FwdTraits {
     static constexpr int THREADS = 384;
     // Register split: warpgroup 0 (producer, MMA issuer) lowers to REGS_LOW,
     // the two softmax warpgroups raise to REGS_HIGH.  128*80 + 256*208 = 63488
-    // <= 384 threads * 168 registers = 64512, the pool the block is launched
-    // with; the host refuses to launch unless the compiled register count
-    // provides that pool.
+    // (decoupled: 128*64 + 256*216 = 63488, the waits for the previous P.V
+    // product need the extra softmax registers) <= 384 threads * 168
+    // registers = 64512, the pool the block is launched with; the host
+    // refuses to launch unless the compiled register count provides that pool.
     static constexpr uint32_t REGS_LAUNCH = 168;
-    static constexpr uint32_t REGS_LOW = 80;
-    static constexpr uint32_t REGS_HIGH = 208;
+    static constexpr uint32_t REGS_LOW = DEC ? 64 : 80;
+    static constexpr uint32_t REGS_HIGH = DEC ? 216 : 208;
     static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= THREADS * REGS_LAUNCH, "register split");
     static constexpr uint32_t TMEM_COLS = 512;
     // S0, S1 [0, 256); decoupled: P0, P1 [256, 384) (bf16, two per column),
