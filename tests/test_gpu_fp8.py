@@ -117,6 +117,27 @@ def test_fp8_forward(fl, oracle, B, H, Lq, Lk, causal, wl, wr):
     assert int(counter.item()) == B * H * c["visited"]
 
 
+@pytest.mark.parametrize("causal,wl,wr", [(True, -1, -1), (False, 200, 200)])
+def test_fp8_rescale_stress(fl, oracle, causal, wl, wr):
+    """Scores spread over a wide range (Q scaled by 6 before quantizing): the
+    reference max of the recurrence moves past its slack of 4 many times and
+    O is rescaled in TMEM; against the oracle's FP8 recurrence on the same
+    codes."""
+    d, L = 128, 1024
+    q, k, v = synth.random_qkv(1, 2, L, L, d, "bf16", seed=77 + max(wl, 0))
+    q = (q.float() * 6.0).to(torch.bfloat16)
+    q8, k8, vt8, qs, ks, vs = _quantized(fl, q, k, v)
+    o, lse = fl.attn_fwd_fp8(q8, k8, vt8, qs, ks, vs, scale=d ** -0.5, causal=causal, window_left=wl,
+                             window_right=wr)
+    torch.cuda.synchronize()
+    assert fl.fattn_device_status() == 0
+    v8n = np.ascontiguousarray(np.swapaxes(vt8.cpu().numpy()[..., :L], 2, 3))
+    o_ref, lse_ref = oracle.attn_fp8(q8.cpu().numpy(), k8.cpu().numpy(), v8n, qs.cpu().numpy(), ks.cpu().numpy(),
+                                     vs.cpu().numpy(), d ** -0.5, causal, wl, wr)
+    compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, BF16_O_MAXABS, BF16_O_RELL2, LSE_ABS,
+            label=f"fp8 rescale stress {causal, wl, wr}")
+
+
 def test_fp8_full_size_causal_4k_sampled_heads(fl, oracle):
     """The causal 4 x 16 x 4096 workload through the GPU quantizer and the FP8
     forward; two heads checked against the oracle's FP8 recurrence."""
