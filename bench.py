@@ -44,6 +44,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 METRIC = "attention fwd TFLOP/s (in-mask FLOPs) & % bf16 tensor peak; decode HBM GB/s"
 HEADLINE = "causal_4k"
 HEADLINE_D64 = "causal_4k_d64"
+WINDOW_D64 = "window_bidir_32k_d64"
 HEADLINE_REPEATS = 5
 DECODE = "decode_32k"
 EXTRA = ["window_bidir_32k", "window_causal_32k", "causal_64k_qscale"]
@@ -786,6 +787,8 @@ def run_ours(args, world, rank, local):
     if not args.no_extra and not args.no_d64:
         extra[HEADLINE_D64] = prefill_line(world, rank, dev, fattn, peaks, peak_src, HEADLINE_D64,
                                            max(3, min(args.steps, 20)))
+        extra[WINDOW_D64] = prefill_line(world, rank, dev, fattn, peaks, peak_src, WINDOW_D64,
+                                         max(3, min(args.steps, 10)))
     if not args.no_extra and not args.no_windows:
         for name in EXTRA:
             extra[name] = prefill_line(world, rank, dev, fattn, peaks, peak_src, name, max(3, min(args.steps, 10)))
@@ -874,7 +877,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-windows", action="store_true", help="skip the window and 64K lines (keeps varlen)")
     ap.add_argument("--no-varlen", action="store_true", help="skip the packed varlen line")
-    ap.add_argument("--no-d64", action="store_true", help="skip the d = 64 prefill line")
+    ap.add_argument("--no-d64", action="store_true", help="skip the d = 64 prefill lines")
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-fp8", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

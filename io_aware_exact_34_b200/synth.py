@@ -66,6 +66,9 @@ WORKLOADS = {
     # sliding window n = 32768, bidirectional |i - j| <= 2048
     "window_bidir_32k": Workload("window_bidir_32k", "prefill", 1, 32, 32768, 32768, 128,
                                  "bf16", window_left=2048, window_right=2048, seed=3),
+    # the same bidirectional window at head dim 64
+    "window_bidir_32k_d64": Workload("window_bidir_32k_d64", "prefill", 1, 32, 32768, 32768, 64,
+                                     "bf16", window_left=2048, window_right=2048, seed=9),
     # sliding window n = 32768, causal left window j in [i - 4096, i]
     "window_causal_32k": Workload("window_causal_32k", "prefill", 1, 32, 32768, 32768, 128,
                                   "bf16", causal=True, window_left=4096, window_right=0, seed=3),

@@ -192,7 +192,8 @@ def test_causal_4k_full(fl, oracle, name):
     compare(o, lse, o_ref, lse_ref, BF16_O_MAXABS, BF16_O_RELL2, label=name)
 
 
-@pytest.mark.parametrize("name", ["window_bidir_32k", "window_causal_32k", "causal_64k_qscale"])
+@pytest.mark.parametrize("name", ["window_bidir_32k", "window_causal_32k", "causal_64k_qscale",
+                                  "window_bidir_32k_d64"])
 def test_long_workloads_sampled(fl, oracle, name):
     """Sliding-window and long causal workloads at full size: the GPU runs
     the whole problem; the oracle checks one full head plus stratified rows of
